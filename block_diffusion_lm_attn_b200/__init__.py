@@ -1,0 +1,177 @@
+"""Python binding of libbdattn.so, the B200 block-diffusion attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/bd_attn.h``.  There is no
+CPU or PyTorch fallback; if the library is missing or cannot be loaded,
+every call raises.
+
+Two layers:
+  * ``bd_attn_fwd`` / ``bd_attn_decode`` / ``bd_attn_decode_workspace_bytes``
+    / ``bd_attn_get_device_status`` / ``bd_attn_status_string`` take the C
+    arguments one to one (device pointers as ints, stream as an int handle)
+    and return the status code.
+  * ``fwd`` / ``decode`` take torch CUDA tensors, check shapes, allocate the
+    outputs if not given, call the C entry point on the current stream and
+    raise ``BdAttnError`` on a non-OK status.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbdattn.so")
+
+BD_OK = 0
+BD_ERR_INVALID_ARG = 1
+BD_ERR_UNSUPPORTED = 2
+BD_ERR_CUDA = 3
+BD_ERR_DEVICE_TIMEOUT = 4
+
+EXPORTED = ("bd_attn_fwd", "bd_attn_decode", "bd_attn_decode_workspace_bytes",
+            "bd_attn_get_device_status", "bd_attn_status_string")
+
+
+class BdAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s failed: %s (status %d)" %
+                         (what, bd_attn_status_string(status), status))
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libbdattn.so (built by ``build.build()``); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(
+            "libbdattn.so not built at %s: run "
+            "`python -m block_diffusion_lm_attn_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.bd_attn_fwd.restype = i
+    lib.bd_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    lib.bd_attn_decode.restype = i
+    lib.bd_attn_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i,
+                                   vp, i, vp, ctypes.c_size_t]
+    lib.bd_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.bd_attn_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    lib.bd_attn_get_device_status.restype = i
+    lib.bd_attn_get_device_status.argtypes = [vp]
+    lib.bd_attn_status_string.restype = ctypes.c_char_p
+    lib.bd_attn_status_string.argtypes = [i]
+    _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------------------
+# one-to-one C entry points
+
+
+def bd_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, b, d, scale, stream):
+    return load().bd_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, L, b, d, scale,
+                              stream)
+
+
+def bd_attn_decode(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq, Hkv,
+                   b, d, intra_block_mode, stream, S_cap, workspace,
+                   workspace_bytes):
+    return load().bd_attn_decode(q_blk, k_cache, v_cache, cache_len, out, lse,
+                                 B, Hq, Hkv, b, d, intra_block_mode, stream,
+                                 S_cap, workspace, workspace_bytes)
+
+
+def bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap):
+    return int(load().bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap))
+
+
+def bd_attn_get_device_status(stream):
+    return load().bd_attn_get_device_status(stream)
+
+
+def bd_attn_status_string(status):
+    return load().bd_attn_status_string(status).decode()
+
+
+# ---------------------------------------------------------------------------
+# torch-tensor conveniences
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def fwd(q, k, v, L: int, b: int, scale: float | None = None, out=None,
+        lse=None, stream=None):
+    """Training/prefill block-diffusion attention on CUDA tensors.
+
+    q [B,Hq,2L,d], k, v [B,Hkv,2L,d] bf16 contiguous.  Returns (out, lse)."""
+    import torch
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if N != 2 * L or tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    for t in (q, k, v):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
+    if scale is None:
+        scale = d ** -0.5
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    st = bd_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                     lse.data_ptr(), B, Hq, Hkv, L, b, d, float(scale),
+                     _stream_handle(stream))
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_attn_fwd")
+    return out, lse
+
+
+def decode(q_blk, k_cache, v_cache, cache_len, mode: int, out=None, lse=None,
+           workspace=None, stream=None):
+    """Block-decode attention on CUDA tensors.
+
+    q_blk [B,Hq,b,d]; k_cache, v_cache [B,Hkv,S_cap,d] bf16; cache_len int32
+    [B] on the device; mode 0 bidirectional, 1 causal.  ``workspace`` is an
+    optional uint8 CUDA tensor of at least ``workspace_bytes(...)`` bytes
+    (None: the library's own per-device buffer).  Returns (out, lse)."""
+    import torch
+    B, Hq, b, d = q_blk.shape
+    Hkv, S_cap = k_cache.shape[1], k_cache.shape[2]
+    if tuple(k_cache.shape) != (B, Hkv, S_cap, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if not (cache_len.is_cuda and cache_len.dtype == torch.int32
+            and cache_len.numel() == B):
+        raise ValueError("cache_len must be an int32 CUDA tensor of B entries")
+    for t in (q_blk, k_cache, v_cache):
+        if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()):
+            raise ValueError("q_blk and caches must be contiguous bf16 CUDA")
+    if out is None:
+        out = torch.empty_like(q_blk)
+    if lse is None:
+        lse = torch.empty((B, Hq, b), device=q_blk.device, dtype=torch.float32)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    st = bd_attn_decode(q_blk.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(),
+                        cache_len.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                        B, Hq, Hkv, b, d, int(mode), _stream_handle(stream),
+                        S_cap, ws_ptr, ws_bytes)
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_attn_decode")
+    return out, lse
+
+
+def workspace_bytes(B, Hq, Hkv, b, d, S_cap) -> int:
+    return bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap)
+
+
+def device_status(stream=None) -> int:
+    return bd_attn_get_device_status(_stream_handle(stream))

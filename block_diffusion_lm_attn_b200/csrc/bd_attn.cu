@@ -1,0 +1,266 @@
+// C-ABI entry points of libbdattn.so: argument validation, launch planning
+// and kernel launches on the caller's stream.  See include/bd_attn.h for the
+// contract of each call.
+#include "bd_attn.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "attn_mma.cuh"
+#include "bd_common.cuh"
+
+namespace {
+
+using bd::bf16;
+
+constexpr int kNumSMs = 148; // B200; used to size split-KV grids
+
+inline bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline bool supported_d(int d) { return d == 32 || d == 64 || d == 128; }
+
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// Split-KV plan for block decode: keys [0, S_cap) of every (batch, kv-head)
+// are cut into `nsplit` chunks of `chunk` keys (a multiple of 64), enough to
+// give the grid a few CTAs per SM.  A pure function of the sizes, so the
+// workspace query and the launch agree without a device round trip.
+struct DecodePlan {
+    int row_tiles, nsplit, chunk;
+    size_t rows_all, o_bytes, lse_bytes, total_bytes;
+};
+
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
+                 DecodePlan &pl)
+{
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap < b ||
+        Hq % Hkv != 0)
+        return false;
+    const long long rows = (long long)(Hq / Hkv) * b;
+    pl.row_tiles = (int)cdiv(rows, bd::kMmaBM);
+    const long long units = (long long)B * Hkv * pl.row_tiles;
+    const long long target = 4LL * kNumSMs;
+    long long ns = cdiv(target, units);
+    const long long max_ns = cdiv(S_cap, 256);
+    if (ns > max_ns) ns = max_ns;
+    if (ns < 1) ns = 1;
+    long long chunk = cdiv(cdiv(S_cap, ns), 64) * 64;
+    pl.chunk = (int)chunk;
+    pl.nsplit = (int)cdiv(S_cap, chunk);
+    pl.rows_all = (size_t)B * Hq * b;
+    pl.o_bytes = round256((size_t)pl.nsplit * pl.rows_all * d * sizeof(float));
+    pl.lse_bytes = round256((size_t)pl.nsplit * pl.rows_all * sizeof(float));
+    pl.total_bytes = pl.o_bytes + pl.lse_bytes;
+    return true;
+}
+
+// Per-device cache of the internal decode workspace (workspace == NULL).
+struct InternalWorkspace {
+    std::mutex mu;
+    void *ptr[64] = {};
+    size_t bytes[64] = {};
+};
+InternalWorkspace g_ws;
+
+bd_status get_internal_workspace(size_t need, void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return BD_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_ws.mu);
+    if (g_ws.bytes[dev] < need) {
+        if (g_ws.ptr[dev])
+            cudaFree(g_ws.ptr[dev]);
+        g_ws.ptr[dev] = nullptr;
+        g_ws.bytes[dev] = 0;
+        if (cudaMalloc(&g_ws.ptr[dev], need) != cudaSuccess) {
+            g_ws.ptr[dev] = nullptr;
+            return BD_ERR_CUDA;
+        }
+        g_ws.bytes[dev] = need;
+    }
+    *out = g_ws.ptr[dev];
+    return BD_OK;
+}
+
+template <class K> bd_status set_smem(K kernel, int bytes)
+{
+    // idempotent; cheap enough to repeat per call
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             bytes) != cudaSuccess)
+        return BD_ERR_CUDA;
+    return BD_OK;
+}
+
+template <int D>
+bd_status launch_fwd_mma(const bd::MmaParams &p, cudaStream_t st)
+{
+    auto kern = bd::bd_mma_attn_kernel<D, 0>;
+    constexpr int smem = bd::mma_smem_bytes<D>();
+    if (set_smem(kern, smem) != BD_OK)
+        return BD_ERR_CUDA;
+    dim3 grid(2 * p.qtiles, p.B * p.Hq);
+    kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+template <int D>
+bd_status launch_decode_mma(const bd::MmaParams &p, const DecodePlan &pl,
+                            cudaStream_t st)
+{
+    auto kern = bd::bd_mma_attn_kernel<D, 1>;
+    constexpr int smem = bd::mma_smem_bytes<D>();
+    if (set_smem(kern, smem) != BD_OK)
+        return BD_ERR_CUDA;
+    dim3 grid(pl.nsplit, pl.row_tiles, p.B * p.Hkv);
+    kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
+    if (cudaGetLastError() != cudaSuccess)
+        return BD_ERR_CUDA;
+    const int rows_all = p.B * p.Hq * p.b;
+    bd::bd_decode_combine_kernel<D><<<(rows_all + 7) / 8, 256, 0, st>>>(p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+} // namespace
+
+extern "C" {
+
+const char *bd_attn_status_string(bd_status s)
+{
+    switch (s) {
+    case BD_OK: return "ok";
+    case BD_ERR_INVALID_ARG: return "invalid argument";
+    case BD_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BD_ERR_CUDA: return "CUDA error";
+    case BD_ERR_DEVICE_TIMEOUT:
+        return "device-side check failed (bounded wait ran out or bad size)";
+    }
+    return "unknown status";
+}
+
+bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                      float *lse, int B, int Hq, int Hkv, int L, int b, int d,
+                      float scale, cudaStream_t stream)
+{
+    if (!q || !k || !v || !out || !lse)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(lse))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || b <= 0 || d <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || L % b != 0)
+        return BD_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    if ((long long)B * Hq > 65535LL || 2LL * L * (long long)B * Hq * d > (1LL << 40))
+        return BD_ERR_UNSUPPORTED;
+
+    bd::MmaParams p = {};
+    p.q = static_cast<const bf16 *>(q);
+    p.k = static_cast<const bf16 *>(k);
+    p.v = static_cast<const bf16 *>(v);
+    p.out = static_cast<bf16 *>(out);
+    p.lse = lse;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
+    p.nkeys = 2 * L;
+    p.qtiles = (int)cdiv(L, bd::kMmaBM);
+    p.scale_log2 = scale * bd::kLog2e;
+    switch (d) {
+    case 32: return launch_fwd_mma<32>(p, stream);
+    case 64: return launch_fwd_mma<64>(p, stream);
+    default: return launch_fwd_mma<128>(p, stream);
+    }
+}
+
+size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int d,
+                                      int S_cap)
+{
+    DecodePlan pl;
+    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
+        return 0;
+    return pl.total_bytes;
+}
+
+bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
+                         const void *v_cache, const int32_t *cache_len,
+                         void *out, float *lse, int B, int Hq, int Hkv, int b,
+                         int d, int intra_block_mode, cudaStream_t stream,
+                         int S_cap, void *workspace, size_t workspace_bytes)
+{
+    if (!q_blk || !k_cache || !v_cache || !cache_len || !out || !lse)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(out) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || S_cap < b)
+        return BD_ERR_INVALID_ARG;
+    if (intra_block_mode != 0 && intra_block_mode != 1)
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    DecodePlan pl;
+    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
+        return BD_ERR_INVALID_ARG;
+    if ((long long)B * Hkv > 65535LL || pl.row_tiles > 65535)
+        return BD_ERR_UNSUPPORTED;
+    if (workspace) {
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+            workspace_bytes < pl.total_bytes)
+            return BD_ERR_INVALID_ARG;
+    } else {
+        bd_status st = get_internal_workspace(pl.total_bytes, &workspace);
+        if (st != BD_OK)
+            return st;
+    }
+
+    bd::MmaParams p = {};
+    p.q = static_cast<const bf16 *>(q_blk);
+    p.k = static_cast<const bf16 *>(k_cache);
+    p.v = static_cast<const bf16 *>(v_cache);
+    p.out = static_cast<bf16 *>(out);
+    p.lse = lse;
+    p.part_o = static_cast<float *>(workspace);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                           pl.o_bytes);
+    p.cache_len = cache_len;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
+    p.nkeys = S_cap;
+    p.mode = intra_block_mode;
+    p.chunk = pl.chunk;
+    p.nsplit = pl.nsplit;
+    p.scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
+    switch (d) {
+    case 32: return launch_decode_mma<32>(p, pl, stream);
+    case 64: return launch_decode_mma<64>(p, pl, stream);
+    default: return launch_decode_mma<128>(p, pl, stream);
+    }
+}
+
+bd_status bd_attn_get_device_status(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess)
+        return BD_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, bd::g_status_word, sizeof word) !=
+        cudaSuccess)
+        return BD_ERR_CUDA;
+    if (word != 0 &&
+        cudaMemcpyToSymbol(bd::g_status_word, &zero, sizeof zero) != cudaSuccess)
+        return BD_ERR_CUDA;
+    return word ? BD_ERR_DEVICE_TIMEOUT : BD_OK;
+}
+
+} // extern "C"

@@ -1,0 +1,153 @@
+/*
+ * bd_attn.h -- C ABI of the B200 (sm_100a) block-diffusion attention library
+ * (libbdattn.so).
+ *
+ * Two operations, both exact masked softmax attention with a natural-log
+ * log-sum-exp side output:
+ *
+ *   bd_attn_fwd     training / prefill form over the sequence [x_t ; x_0].
+ *   bd_attn_decode  block-decode form: a block of b noisy queries over a
+ *                   clean KV cache plus the block itself.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous
+ *     row-major, 16-byte aligned.  bf16 tensors are IEEE bfloat16 bit patterns.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and return right after the launch.  They never synchronise the
+ *     host, never allocate (except bd_attn_decode with workspace == NULL, see
+ *     there) and never free.
+ *   - No exception or abort crosses the ABI: every error is a bd_status.
+ *     Argument errors are detected on the host before anything is launched;
+ *     nothing is written to any output in that case.
+ *   - Grouped-query attention: q-head h reads kv-head h / (Hq / Hkv).
+ *   - lse is ln( sum over visible keys of exp(scale * q.k) ).
+ */
+#ifndef BD_ATTN_H
+#define BD_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+#if defined(__GNUC__)
+#define BD_API __attribute__((visibility("default")))
+#else
+#define BD_API
+#endif
+
+typedef enum {
+    BD_OK = 0,
+    BD_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size or mode */
+    BD_ERR_UNSUPPORTED = 2,     /* valid request this build does not handle */
+    BD_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
+    BD_ERR_DEVICE_TIMEOUT = 4   /* a bounded device wait ran out, or a
+                                   device-side range check failed */
+} bd_status;
+
+/*
+ * Training / prefill block-diffusion attention.
+ *
+ * Defines: the three-part mask of "Nemotron-Labs-Diffusion-8B-Base 3x decoding
+ * speed-up" (doido.pw), section 1 "Block Diffusion Attention" -- block
+ * diagonal M_BD, offset block-causal M_OBC, block-causal M_BC -- read with the
+ * BDLM objective of "LLaDA2.0-Uni" (discuss.pytorch.kr), section "Training
+ * objective and loss function", eq. L_BDLM, which predicts x_{0,k} from
+ * x_{0,<k} and x_{t,k} with K = L_total / L_B blocks.
+ *
+ * Each (batch, head) slice is a sequence of N = 2L rows: rows 0..L-1 are the
+ * noisy tokens x_t, rows L..2L-1 the clean tokens x_0, each half cut into L/b
+ * blocks of b rows.  A noisy row of block k sees the noisy rows of block k
+ * (bidirectionally) and the clean rows of blocks < k; a clean row of block k
+ * sees the clean rows of blocks <= k; no row sees a noisy row of another
+ * block, and clean rows see no noisy row.
+ *
+ *   q    [B, Hq,  2L, d] bf16      (read)
+ *   k, v [B, Hkv, 2L, d] bf16      (read)
+ *   out  [B, Hq,  2L, d] bf16      (written: softmax(scale q k^T) v, rounded
+ *                                   to nearest even)
+ *   lse  [B, Hq,  2L]    fp32      (written)
+ *   scale: softmax scale applied to q.k (typically 1/sqrt(d)); finite, > 0.
+ *
+ * Errors: BD_ERR_INVALID_ARG for a null or non-16-byte-aligned pointer, any
+ * size <= 0, Hq % Hkv != 0, L % b != 0, or a non-finite/non-positive scale;
+ * BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA if the launch
+ * fails.
+ */
+BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                      float *lse, int B, int Hq, int Hkv, int L, int b, int d,
+                      float scale, struct CUstream_st *stream);
+
+/*
+ * Block-decode block-diffusion attention.
+ *
+ * Defines: a block of b noisy queries attends to the cached clean prefix and
+ * to its own block, bidirectionally while denoising a draft and causally when
+ * verifying it against the same cache: "Nemotron-Labs-Diffusion-8B-Base 3x
+ * decoding speed-up", section 2 "Linear Speculative Decoding";
+ * "Nemotron-Labs-Diffusion-VLM-8B", section "Multi-mode decoding";
+ * "Nemotron-Labs-Diffusion-3B", section "What it is" (guess a run of tokens
+ * and check them in the same cache memory).
+ *
+ * The caller has already written the block's own K/V into the caches at
+ * positions cache_len[i] .. cache_len[i]+b-1; cache_len counts the clean
+ * prefix only.  Block row j of sequence i sees cache positions
+ * 0 .. cache_len[i]-1 and block positions cache_len[i]+j' for every j' < b
+ * (intra_block_mode 0, bidirectional denoise) or every j' <= j
+ * (intra_block_mode 1, causal verify).  Softmax scale is 1/sqrt(d).
+ *
+ *   q_blk            [B, Hq, b, d]        bf16 (read)
+ *   k_cache, v_cache [B, Hkv, S_cap, d]   bf16 (read; rows beyond
+ *                                               cache_len[i]+b never read)
+ *   cache_len        [B] int32, DEVICE memory (read on the device only, so
+ *                    the call never waits for the host and can be captured in
+ *                    a CUDA graph)
+ *   out              [B, Hq, b, d]        bf16 (written)
+ *   lse              [B, Hq, b]           fp32 (written)
+ *   S_cap            row capacity of the caches (>= b)
+ *   workspace        device scratch of at least
+ *                    bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap)
+ *                    bytes, 256-byte aligned, used for the split-KV partial
+ *                    results; its contents on entry do not matter.  NULL
+ *                    makes the library use a buffer it allocates once per
+ *                    device and keeps (that first call allocates, so it must
+ *                    not be inside a stream capture).
+ *
+ * Errors: BD_ERR_INVALID_ARG for a null or misaligned pointer, any size <= 0,
+ * Hq % Hkv != 0, S_cap < b, intra_block_mode not 0/1, or a workspace smaller
+ * than required; BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA
+ * if the launch (or the internal workspace allocation) fails.  A cache_len[i]
+ * outside [0, S_cap - b] is caught on the device: that sequence's rows are
+ * written as NaN with lse NaN, and the device status word (see
+ * bd_attn_get_device_status) records BD_ERR_DEVICE_TIMEOUT.
+ */
+BD_API bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
+                         const void *v_cache, const int32_t *cache_len,
+                         void *out, float *lse, int B, int Hq, int Hkv, int b,
+                         int d, int intra_block_mode,
+                         struct CUstream_st *stream, int S_cap,
+                         void *workspace, size_t workspace_bytes);
+
+/* Bytes of scratch bd_attn_decode needs for these sizes (0 on bad sizes).
+ * Pure host arithmetic; needs no GPU. */
+BD_API size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int d,
+                                      int S_cap);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: BD_OK, or BD_ERR_DEVICE_TIMEOUT if a kernel gave up a
+ * bounded wait or rejected a device-resident size since the last call;
+ * BD_ERR_CUDA if the synchronisation itself failed. */
+BD_API bd_status bd_attn_get_device_status(struct CUstream_st *stream);
+
+/* Static, NUL-terminated description of a status code. */
+BD_API const char *bd_attn_status_string(bd_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BD_ATTN_H */

@@ -1,0 +1,111 @@
+"""The C-ABI library builds, loads and exports every declared entry point,
+and rejects bad arguments on the host (no GPU needed: nothing is launched)."""
+import os
+import re
+
+import pytest
+
+import block_diffusion_lm_attn_b200 as bd
+from block_diffusion_lm_attn_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return bd.load()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names += re.findall(r"\b(bd_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(bd.EXPORTED) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert bd.bd_attn_status_string(s)
+    assert bd.bd_attn_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes(lib):
+    assert bd.bd_attn_decode_workspace_bytes(16, 32, 8, 32, 128, 8224) > 0
+    assert bd.bd_attn_decode_workspace_bytes(0, 32, 8, 32, 128, 8224) == 0
+    assert bd.bd_attn_decode_workspace_bytes(1, 6, 4, 32, 128, 64) == 0
+    assert bd.bd_attn_decode_workspace_bytes(1, 4, 4, 32, 128, 16) == 0
+    w = bd.bd_attn_decode_workspace_bytes(16, 32, 8, 32, 128, 8224)
+    assert w % 256 == 0
+
+
+A = 1 << 20  # a 16-byte-aligned fake address; never dereferenced
+
+
+def fwd_args(**kw):
+    a = dict(q=A, k=A, v=A, out=A, lse=A, B=1, Hq=2, Hkv=2, L=64, b=8, d=32,
+             scale=0.17, stream=None)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), bd.BD_ERR_INVALID_ARG),
+    (dict(lse=None), bd.BD_ERR_INVALID_ARG),
+    (dict(k=A + 8), bd.BD_ERR_INVALID_ARG),
+    (dict(out=A + 2), bd.BD_ERR_INVALID_ARG),
+    (dict(B=0), bd.BD_ERR_INVALID_ARG),
+    (dict(L=-64), bd.BD_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), bd.BD_ERR_INVALID_ARG),
+    (dict(L=60, b=8), bd.BD_ERR_INVALID_ARG),
+    (dict(scale=0.0), bd.BD_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), bd.BD_ERR_INVALID_ARG),
+    (dict(d=96), bd.BD_ERR_UNSUPPORTED),
+    (dict(d=256), bd.BD_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects(lib, kw, status):
+    assert bd.bd_attn_fwd(**fwd_args(**kw)) == status
+
+
+def dec_args(**kw):
+    a = dict(q_blk=A, k_cache=A, v_cache=A, cache_len=A, out=A, lse=A, B=2,
+             Hq=4, Hkv=2, b=8, d=64, intra_block_mode=0, stream=None, S_cap=64,
+             workspace=A, workspace_bytes=1 << 30)
+    a.update(kw)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cache_len=None), bd.BD_ERR_INVALID_ARG),
+    (dict(v_cache=A + 4), bd.BD_ERR_INVALID_ARG),
+    (dict(cache_len=A + 2), bd.BD_ERR_INVALID_ARG),
+    (dict(Hq=3), bd.BD_ERR_INVALID_ARG),
+    (dict(S_cap=4), bd.BD_ERR_INVALID_ARG),
+    (dict(intra_block_mode=2), bd.BD_ERR_INVALID_ARG),
+    (dict(b=0), bd.BD_ERR_INVALID_ARG),
+    (dict(workspace_bytes=16), bd.BD_ERR_INVALID_ARG),
+    (dict(workspace=A + 16), bd.BD_ERR_INVALID_ARG),
+    (dict(d=80), bd.BD_ERR_UNSUPPORTED),
+])
+def test_decode_rejects(lib, kw, status):
+    assert bd.bd_attn_decode(**dec_args(**kw)) == status
+
+
+def test_product_path_does_not_touch_the_oracle():
+    """The library sources and the binding never name the oracle."""
+    pkg = os.path.join(ROOT, "block_diffusion_lm_attn_b200")
+    for dp, _, fns in os.walk(pkg):
+        for fn in fns:
+            if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                txt = open(os.path.join(dp, fn)).read()
+                assert "oracle" not in txt.lower(), fn
