@@ -175,3 +175,17 @@ def workspace_bytes(B, Hq, Hkv, b, d, S_cap) -> int:
 
 def device_status(stream=None) -> int:
     return bd_attn_get_device_status(_stream_handle(stream))
+
+
+def bd_attn_decode_noalloc(q_blk, k_cache, v_cache, cache_len, out, lse, B,
+                           Hq, Hkv, b, d, intra_block_mode, stream, S_cap):
+    """One-to-one binding of the C entry point that decodes without
+    allocating: its split-KV scratch is a fixed array inside the library
+    (see include/bd_attn.h), for callers that cannot allocate device memory
+    at decode time."""
+    fn = load().bd_attn_decode_noalloc
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    fn.restype = i
+    fn.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, i]
+    return fn(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq, Hkv, b, d,
+              intra_block_mode, stream, S_cap)

@@ -264,3 +264,95 @@ bd_status bd_attn_get_device_status(cudaStream_t stream)
 }
 
 } // extern "C"
+
+// ---------------------------------------------------------------------------
+// Block decode without allocation: the split-KV scratch is this fixed array
+// in the library's device memory.  Host code must not use the array's name as
+// an address (on the host it is only a stand-in); the device address is
+// looked up once per device with cudaGetSymbolAddress and passed to the
+// kernels.
+
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[BD_ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+struct NoallocScratch {
+    std::mutex mu;
+    void *addr[64] = {};
+};
+NoallocScratch g_noalloc;
+
+// Device address of g_noalloc_scratch on the current device (looked up on
+// the first call for that device, with that device current).
+bd_status noalloc_scratch_address(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return BD_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc.mu);
+    if (!g_noalloc.addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return BD_ERR_CUDA;
+        g_noalloc.addr[dev] = p;
+    }
+    *out = g_noalloc.addr[dev];
+    return BD_OK;
+}
+
+} // namespace
+
+extern "C" bd_status bd_attn_decode_noalloc(
+    const void *q_blk, const void *k_cache, const void *v_cache,
+    const int32_t *cache_len, void *out, float *lse, int B, int Hq, int Hkv,
+    int b, int d, int intra_block_mode, cudaStream_t stream, int S_cap)
+{
+    if (!q_blk || !k_cache || !v_cache || !cache_len || !out || !lse)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(out) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || S_cap < b)
+        return BD_ERR_INVALID_ARG;
+    if (intra_block_mode != 0 && intra_block_mode != 1)
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    DecodePlan pl;
+    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
+        return BD_ERR_INVALID_ARG;
+    if ((long long)B * Hkv > 65535LL || pl.row_tiles > 65535)
+        return BD_ERR_UNSUPPORTED;
+    if (pl.total_bytes > (size_t)BD_ATTN_NOALLOC_SCRATCH_BYTES)
+        return BD_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    bd_status st = noalloc_scratch_address(&scratch);
+    if (st != BD_OK)
+        return st;
+
+    bd::MmaParams p = {};
+    p.q = static_cast<const bf16 *>(q_blk);
+    p.k = static_cast<const bf16 *>(k_cache);
+    p.v = static_cast<const bf16 *>(v_cache);
+    p.out = static_cast<bf16 *>(out);
+    p.lse = lse;
+    p.part_o = static_cast<float *>(scratch);
+    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) +
+                                           pl.o_bytes);
+    p.cache_len = cache_len;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
+    p.nkeys = S_cap;
+    p.mode = intra_block_mode;
+    p.chunk = pl.chunk;
+    p.nsplit = pl.nsplit;
+    p.scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
+    switch (d) {
+    case 32: return launch_decode_mma<32>(p, pl, stream);
+    case 64: return launch_decode_mma<64>(p, pl, stream);
+    default: return launch_decode_mma<128>(p, pl, stream);
+    }
+}

@@ -132,6 +132,44 @@ BD_API bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
                          struct CUstream_st *stream, int S_cap,
                          void *workspace, size_t workspace_bytes);
 
+/* Size of the fixed scratch array bd_attn_decode_noalloc works in. */
+#define BD_ATTN_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * Block decode that never allocates device memory (no counterpart on the
+ * source pages; it exists for callers that cannot allocate).
+ *
+ * Some callers cannot call cudaMalloc at the point where they decode: a
+ * serving loop whose device memory is owned entirely by another allocator
+ * (a framework's caching allocator, a fixed memory budget), code running
+ * inside a stream capture where allocation is not allowed, or real-time code
+ * that forbids allocation after start-up.  This call computes exactly what
+ * bd_attn_decode computes, with the same arguments, layouts and errors, but
+ * takes no workspace: its split-KV scratch is a fixed array of
+ * BD_ATTN_NOALLOC_SCRATCH_BYTES bytes compiled into the library's device
+ * code.  Every GPU on which the library's kernels are loaded holds that array
+ * until the process exits.
+ *
+ * - The first call on a device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.
+ * - Sizes whose scratch, bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d,
+ *   S_cap), exceeds BD_ATTN_NOALLOC_SCRATCH_BYTES are rejected with
+ *   BD_ERR_UNSUPPORTED before anything is launched.
+ * - All calls share the one array and it keeps whatever the last call left
+ *   there; nothing in it needs to start at zero.  Calls whose kernels overlap
+ *   on the GPU (for example on two streams without ordering between them)
+ *   race on the array and give wrong results: order them on one stream or
+ *   with events.
+ * - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+BD_API bd_status bd_attn_decode_noalloc(const void *q_blk, const void *k_cache,
+                                        const void *v_cache,
+                                        const int32_t *cache_len, void *out,
+                                        float *lse, int B, int Hq, int Hkv,
+                                        int b, int d, int intra_block_mode,
+                                        struct CUstream_st *stream, int S_cap);
+
 /* Bytes of scratch bd_attn_decode needs for these sizes (0 on bad sizes).
  * Pure host arithmetic; needs no GPU. */
 BD_API size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int d,
