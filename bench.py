@@ -38,12 +38,13 @@ import bd_inputs  # noqa: E402
 METRIC = ("BD-attn fwd TFLOP/s (unmasked FLOPs) & block-decode HBM GB/s, "
           "% of roofline")
 L2_FLUSH_BYTES = 256 << 20
-# dram__bytes_read.sum + dram__bytes_write.sum of one fwd launch on the
-# training shape, from the ncu capture summarised in
-# profiles/fwd_kernel_training_shape.md; None until that capture matches
-# the current kernel.
-FWD_TRAFFIC_BYTES = None
-DECODE_TRAFFIC_BYTES = None
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
+# kernel, from the ncu captures summarised under profiles/
+# (bd_mma_attn_kernel_fwd_training_shape.md,
+# bd_mma_attn_kernel_decode_denoise.md); None whenever the kernel has changed
+# since those counters were taken.
+FWD_TRAFFIC_BYTES = 305149696
+DECODE_TRAFFIC_BYTES = 576815104
 
 
 def fwd_flops(s) -> int:
@@ -193,6 +194,30 @@ def timed_steps(fn, steps, warmup, flush, world, sampler=None):
     return max_over_ranks(total, world)
 
 
+def run_e2e(bd, s, q, k, v, qd, kd, vd, out, lse, flush, world, steps):
+    """The same call through the public API with host buffers: pinned-host
+    -> device copies of q, k, v and device -> pinned-host copies of out and
+    lse are inside the timed region of every step."""
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        bd.fwd(qd, kd, vd, s.L, s.b, s.scale, out=out, lse=lse)
+        outh.copy_(out, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    ms = timed_steps(e2e_step, steps, 3, flush, world) / steps
+    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+    return {"value": round(world * fwd_flops(s) / (ms * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 4)}
+
+
 def run_ours(args):
     import block_diffusion_lm_attn_b200 as bd
     world, rank, local = dist_setup(args.gpus)
@@ -206,52 +231,41 @@ def run_ours(args):
     sampler = ClockSampler(gpu_id)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sampler.start()
+    only = args.only
+    rows = {}
+    n_launch = 0
+    value = ms = fwd_kernel_tflops = None
+    e2e = None
+    s = bd_inputs.FWD_TRAIN
 
     # ---- headline: training shape, one bd_attn_fwd per step
-    s = bd_inputs.FWD_TRAIN
-    q, k, v = bd_inputs.fwd_inputs_for(s)
-    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
-    out = torch.empty_like(qd)
-    lse = torch.empty((s.B, s.Hq, 2 * s.L), device=dev, dtype=torch.float32)
+    if only in ("all", "fwd"):
+        q, k, v = bd_inputs.fwd_inputs_for(s)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        out = torch.empty_like(qd)
+        lse = torch.empty((s.B, s.Hq, 2 * s.L), device=dev,
+                          dtype=torch.float32)
 
-    def step():
-        bd.fwd(qd, kd, vd, s.L, s.b, s.scale, out=out, lse=lse)
+        def step():
+            bd.fwd(qd, kd, vd, s.L, s.b, s.scale, out=out, lse=lse)
 
-    total_ms = timed_steps(step, args.steps, args.warmup, flush, world, sampler)
-    ms = total_ms / args.steps
-    flops = fwd_flops(s)
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
-    fwd_kernel_tflops = flops / (ms * 1e-3) / 1e12
-
-    # ---- end to end through the public API with host buffers
-    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    outh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        bd.fwd(qd, kd, vd, s.L, s.b, s.scale, out=out, lse=lse)
-        outh.copy_(out, non_blocking=True)
-        lseh.copy_(lse, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 20))
-    e2e_ms = timed_steps(e2e_step, e2e_steps, 2, flush, world) / e2e_steps
-    h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
-    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
-    e2e = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 3),
-           "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
-    del qh, kh, vh, outh, lseh, qd, kd, vd, out, lse
-
-    rows = {"fwd_train": {"tflops": round(fwd_kernel_tflops, 2),
-                          "ms": round(ms, 4),
-                          "frac_of_measured_bf16": round(fwd_kernel_tflops / tf_burst, 4)}}
-    n_launch = args.steps  # one fwd kernel per step
+        total_ms = timed_steps(step, args.steps, args.warmup, flush, world,
+                               sampler)
+        ms = total_ms / args.steps
+        value = world * fwd_flops(s) * args.steps / (total_ms * 1e-3) / 1e12
+        fwd_kernel_tflops = fwd_flops(s) / (ms * 1e-3) / 1e12
+        n_launch = args.steps  # one fwd kernel per step
+        rows["fwd_train"] = {"tflops": round(fwd_kernel_tflops, 2),
+                             "ms": round(ms, 4),
+                             "frac_of_measured_bf16":
+                                 round(fwd_kernel_tflops / tf_burst, 4)}
+        if only == "all":
+            e2e = run_e2e(bd, s, q, k, v, qd, kd, vd, out, lse, flush, world,
+                          max(3, min(args.steps, 20)))
+        del qd, kd, vd, out, lse
 
     # ---- long-context block-size sweep
-    if not args.quick:
+    if only == "all" and not args.quick:
         for bb, sl in sorted(bd_inputs.FWD_LONG.items()):
             q, k, v = bd_inputs.fwd_inputs_for(sl)
             qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
@@ -267,41 +281,46 @@ def run_ours(args):
                              "frac_of_measured_bf16": round(tf / tf_burst, 4)}
             del qd, kd, vd, o, ls
 
-    # ---- block decode workloads
+    # ---- block decode workloads (split-KV kernel + LSE combine per call)
     dec_roof = None
-    for sd in (bd_inputs.DEC_DENOISE, bd_inputs.DEC_VERIFY):
-        q, kc, vc, cl = bd_inputs.decode_inputs_for(sd)
-        qd, kcd, vcd, cld = q.to(dev), kc.to(dev), vc.to(dev), cl.to(dev)
-        o = torch.empty_like(qd)
-        ls = torch.empty((sd.B, sd.Hq, sd.b), device=dev, dtype=torch.float32)
-        nb = bd.workspace_bytes(sd.B, sd.Hq, sd.Hkv, sd.b, sd.d, sd.S_cap)
-        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
-        n = max(5, args.steps // 5)
-        t = timed_steps(lambda: bd.decode(qd, kcd, vcd, cld, sd.mode, out=o,
-                                          lse=ls, workspace=ws),
-                        n, 3, flush, world, sampler) / n
-        nbytes = decode_bytes(sd, cl.tolist())
-        gbs = nbytes / (t * 1e-3) / 1e9
-        rows[sd.name] = {"gbs": round(gbs, 1), "ms": round(t, 4),
-                         "bytes": nbytes,
-                         "frac_of_measured_hbm": round(gbs / hbm, 4),
-                         "frac_of_8tbs": round(gbs / 8000.0, 4)}
-        if sd is bd_inputs.DEC_DENOISE:
-            dec_roof = {"bound": "hbm", "achieved": round(gbs, 1),
-                        "peak": hbm, "unit": "GB/s",
-                        "frac": round(gbs / hbm, 4),
-                        "traffic": DECODE_TRAFFIC_BYTES,
-                        "peak_source": peak_kind,
-                        "kernels": "split-KV + LSE combine"}
-        del qd, kcd, vcd, o, ls, ws
+    if only in ("all", "decode"):
+        for sd in (bd_inputs.DEC_DENOISE, bd_inputs.DEC_VERIFY):
+            q, kc, vc, cl = bd_inputs.decode_inputs_for(sd)
+            qd, kcd, vcd, cld = q.to(dev), kc.to(dev), vc.to(dev), cl.to(dev)
+            o = torch.empty_like(qd)
+            ls = torch.empty((sd.B, sd.Hq, sd.b), device=dev,
+                             dtype=torch.float32)
+            nb = bd.workspace_bytes(sd.B, sd.Hq, sd.Hkv, sd.b, sd.d, sd.S_cap)
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+            n = max(5, args.steps // 5) if only == "all" else args.steps
+            t = timed_steps(lambda: bd.decode(qd, kcd, vcd, cld, sd.mode,
+                                              out=o, lse=ls, workspace=ws),
+                            n, 3, flush, world, sampler) / n
+            nbytes = decode_bytes(sd, cl.tolist())
+            gbs = nbytes / (t * 1e-3) / 1e9
+            rows[sd.name] = {"gbs": round(gbs, 1), "ms": round(t, 4),
+                             "bytes": nbytes,
+                             "frac_of_measured_hbm": round(gbs / hbm, 4),
+                             "frac_of_8tbs": round(gbs / 8000.0, 4)}
+            if sd is bd_inputs.DEC_DENOISE:
+                dec_roof = {"bound": "hbm", "achieved": round(gbs, 1),
+                            "peak": hbm, "unit": "GB/s",
+                            "frac": round(gbs / hbm, 4),
+                            "traffic": DECODE_TRAFFIC_BYTES,
+                            "peak_source": peak_kind,
+                            "kernels": "split-KV + LSE combine"}
+            del qd, kcd, vcd, o, ls, ws
     clocks = sampler.stop()
 
     result = None
     if rank == 0:
         result = {
-            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s",
+            "metric": METRIC,
+            "value": round(value, 3) if value is not None else None,
+            "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms, 5), "higher_is_better": True,
+            "ms_per_step": round(ms, 5) if ms is not None else None,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16; keys x0.5)",
             "config": {"workload": "bd_attn_fwd training shape: B=4 Hq=32 "
@@ -310,19 +329,19 @@ def run_ours(args):
                        "d": s.d, "seq_len": 2 * s.L,
                        "parallelism": "replicas" if world > 1 else "single",
                        "l2": "flushed (256 MB write) before every step"},
-            "roofline": {"bound": "tensor",
-                         "achieved": round(fwd_kernel_tflops, 2),
-                         "peak": tf_burst, "unit": "TFLOP/s",
-                         "frac": round(fwd_kernel_tflops / tf_burst, 4),
-                         "traffic": FWD_TRAFFIC_BYTES,
-                         "peak_source": peak_kind + " bf16 burst"},
+            "roofline": None if fwd_kernel_tflops is None else {
+                "bound": "tensor", "achieved": round(fwd_kernel_tflops, 2),
+                "peak": tf_burst, "unit": "TFLOP/s",
+                "frac": round(fwd_kernel_tflops / tf_burst, 4),
+                "traffic": FWD_TRAFFIC_BYTES,
+                "peak_source": peak_kind + " bf16 burst"},
             "roofline_decode": dec_roof,
             "e2e": e2e,
             "gpu_launches": n_launch,
             "clocks": clocks,
             "rows": rows,
         }
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and only == "all" and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(s, budget_s=args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
@@ -410,6 +429,9 @@ def main():
                     help="skip the long-context sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
+                    help="time only the training-shape fwd or only decode "
+                         "(used for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
