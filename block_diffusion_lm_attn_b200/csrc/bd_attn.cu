@@ -8,7 +8,11 @@
 #include <cstdlib>
 #include <mutex>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "bd_common.cuh"
 
 namespace {
@@ -99,6 +103,60 @@ template <class K> bd_status set_smem(K kernel, int bytes)
     return BD_OK;
 }
 
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
+// point (no link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p,
+                                    cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a row-major bf16 tensor [n2][n1][128]: boxes of 64 columns x
+// 128 rows x 1, 128-byte swizzle, rows beyond n1 read as zero.
+bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
+                      uint64_t n2)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3] = {128, n1, n2};
+    cuuint64_t strides[2] = {128 * 2, 128 * 2 * n1};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                     const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bd_status launch_fwd_tc(const void *q, const void *k, const void *v,
+                        const bd::TcParams &p, cudaStream_t st)
+{
+    CUtensorMap mq, mk, mv;
+    const uint64_t N = 2ull * p.L;
+    if (!make_map_rows128(&mq, q, N, (uint64_t)p.B * p.Hq) ||
+        !make_map_rows128(&mk, k, N, (uint64_t)p.B * p.Hkv) ||
+        !make_map_rows128(&mv, v, N, (uint64_t)p.B * p.Hkv))
+        return BD_ERR_CUDA;
+    auto kern = bd::bd_tc_attn_kernel<0>;
+    if (set_smem(kern, bd::kTcSmemBytes) != BD_OK)
+        return BD_ERR_CUDA;
+    dim3 grid(2 * p.qtiles, p.B * p.Hq);
+    kern<<<grid, bd::kTcThreads, bd::kTcSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
 template <int D>
 bd_status launch_fwd_mma(const bd::MmaParams &p, cudaStream_t st)
 {
@@ -165,6 +223,17 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
     if ((long long)B * Hq > 65535LL || 2LL * L * (long long)B * Hq * d > (1LL << 40))
         return BD_ERR_UNSUPPORTED;
 
+    if (d == 128) {
+        bd::TcParams tp = {};
+        tp.out = static_cast<bf16 *>(out);
+        tp.lse = lse;
+        tp.B = B; tp.Hq = Hq; tp.Hkv = Hkv; tp.L = L; tp.b = b;
+        tp.nkeys = 2 * L;
+        tp.qtiles = (int)cdiv(L, bd::kTcM);
+        tp.scale_log2 = scale * bd::kLog2e;
+        return launch_fwd_tc(q, k, v, tp, stream);
+    }
+
     bd::MmaParams p = {};
     p.q = static_cast<const bf16 *>(q);
     p.k = static_cast<const bf16 *>(k);
@@ -177,8 +246,7 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
     p.scale_log2 = scale * bd::kLog2e;
     switch (d) {
     case 32: return launch_fwd_mma<32>(p, stream);
-    case 64: return launch_fwd_mma<64>(p, stream);
-    default: return launch_fwd_mma<128>(p, stream);
+    default: return launch_fwd_mma<64>(p, stream);
     }
 }
 
@@ -356,3 +424,14 @@ extern "C" bd_status bd_attn_decode_noalloc(
     default: return launch_decode_mma<128>(p, pl, stream);
     }
 }
+
+#ifdef BD_TC_TRACE
+// Debug builds only: point the tensor-core kernel's progress trace at a
+// host-mapped buffer of 8 words per CTA (NULL disables it).
+extern "C" __attribute__((visibility("default"))) int
+bd_debug_set_trace(void *buf)
+{
+    uint32_t *p = static_cast<uint32_t *>(buf);
+    return cudaMemcpyToSymbol(bd::g_tc_trace, &p, sizeof p) == cudaSuccess ? 0 : 1;
+}
+#endif
