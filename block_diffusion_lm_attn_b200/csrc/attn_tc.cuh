@@ -41,6 +41,11 @@ constexpr int kTcM = 128;     // query rows per CTA
 constexpr int kTcN = 128;     // keys per K/V tile
 constexpr int kTcD = 128;     // head dim
 constexpr int kTcStages = 2;  // K/V ring depth
+#ifndef BD_EXP2_EMU
+#define BD_EXP2_EMU 1
+#endif
+// evaluate a quarter of the FULL-tile exponentials with ex2_poly2
+constexpr bool kEmuExp2 = BD_EXP2_EMU != 0;
 constexpr int kTileBytes = kTcN * kTcD * 2;          // 32 KB
 constexpr int kHalfTileBytes = kTileBytes / 2;       // one 64-column box
 #ifdef BD_TC_TRACE
@@ -270,6 +275,98 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn)
 
 // ---------------------------------------------------------------------------
 
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1), one packed instruction.
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1,
+                                      float b0, float b1, float c0, float c1)
+{
+    asm("{\n\t.reg .b64 A, B, C, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "mov.b64 C, {%6, %7};\n\tfma.rn.f32x2 D, A, B, C;\n\t"
+        "mov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) = (a0, a1) + (b0, b1), one packed instruction.
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float a0, float a1,
+                                      float b0, float b1)
+{
+    asm("{\n\t.reg .b64 A, B, D;\n\t"
+        "mov.b64 A, {%2, %3};\n\tmov.b64 B, {%4, %5};\n\t"
+        "add.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, D;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// 2^x for a pair of x <= 8 on the FMA and integer pipes, leaving the
+// special-function unit to the other exponentials of the tile.
+// Cody-Waite reduction: n = round(x) (by adding 1.5 * 2^23, which leaves n
+// in the low mantissa bits), f = x - n in [-1/2, 1/2]; 2^f from the degree-3
+// minimax polynomial (relative error 7.5e-5) fitted by csrc/fit_exp2.py;
+// 2^n applied by adding n to the exponent field.  x is clamped at -126 so
+// the exponent add cannot wrap; such terms are below 2^-126 and do not
+// matter next to the row maximum (2^0 or more).
+__device__ __forceinline__ void ex2_poly2(float &y0, float &y1, float x0,
+                                          float x1)
+{
+    constexpr float kMagic = 12582912.0f; // 1.5 * 2^23
+    constexpr float c0 = 9.999280572e-01f, c1 = 6.932609677e-01f,
+                    c2 = 2.426111251e-01f, c3 = 5.517166853e-02f;
+    x0 = fmaxf(x0, -126.f);
+    x1 = fmaxf(x1, -126.f);
+    float j0, j1, n0, n1, f0, f1, p0, p1;
+    fadd2(j0, j1, x0, x1, kMagic, kMagic);
+    fadd2(n0, n1, j0, j1, -kMagic, -kMagic);
+    ffma2(f0, f1, n0, n1, -1.f, -1.f, x0, x1);
+    ffma2(p0, p1, c3, c3, f0, f1, c2, c2);
+    ffma2(p0, p1, p0, p1, f0, f1, c1, c1);
+    ffma2(p0, p1, p0, p1, f0, f1, c0, c0);
+    y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(j0) << 23));
+    y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(j1) << 23));
+}
+
+// P (bf16, packed over the S columns) and its row sum for one tile.  On
+// FULL tiles (EMU) one pair in four is exponentiated by ex2_poly2; masked
+// entries only occur on the other tiles, where every term goes through
+// ex2.approx so that they stay exactly 0.
+template <bool EMU>
+__device__ __forceinline__ void softmax_p_tile(const float *s, float sl2,
+                                               float nm, uint32_t ts,
+                                               float *rsum)
+{
+#pragma unroll
+    for (int c4 = 0; c4 < kTcN / 32; ++c4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 32; c += 4) {
+            float x0, x1, x2, x3;
+            const int b0 = c4 * 32 + c;
+            ffma2(x0, x1, s[b0], s[b0 + 1], sl2, sl2, nm, nm);
+            ffma2(x2, x3, s[b0 + 2], s[b0 + 3], sl2, sl2, nm, nm);
+            x0 = ex2(x0);
+            x1 = ex2(x1);
+            if (EMU && ((c >> 2) & 1)) {
+                ex2_poly2(x2, x3, x2, x3);
+            } else {
+                x2 = ex2(x2);
+                x3 = ex2(x3);
+            }
+            const int a = (c >> 2) & 1;
+            fadd2(rsum[2 * a], rsum[2 * a + 1], rsum[2 * a], rsum[2 * a + 1], x0, x1);
+            fadd2(rsum[2 * a], rsum[2 * a + 1], rsum[2 * a], rsum[2 * a + 1], x2, x3);
+            pk[c / 2] = pack_bf16x2(x0, x1);
+            pk[c / 2 + 1] = pack_bf16x2(x2, x3);
+        }
+        tmem_st16(ts + c4 * 16, pk);
+    }
+}
+
 // Bits [a, b) of a 32-bit word, with a and b clamped to [0, 32].
 __device__ __forceinline__ uint32_t range_bits(int a, int b)
 {
@@ -360,8 +457,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto bar_vempty = [&](int s) { return bar0 + 8 * (1 + 3 * kTcStages + s); };
     const uint32_t bar_sfull0 = bar0 + 8 * (1 + 4 * kTcStages); // 2 of them
     const uint32_t bar_pfull0 = bar_sfull0 + 16;                // 2 of them
-    const uint32_t bar_odone = bar_pfull0 + 16;
-    const uint32_t bar_final = bar_odone + 8;
+    const uint32_t bar_odone0 = bar_pfull0 + 16;               // 2 of them
+    const uint32_t bar_final = bar_odone0 + 16;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kSmemBar + 200);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + kSmemBar + 208);
 
@@ -387,7 +484,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         mbar_init(bar_sfull0 + 8, 1);
         mbar_init(bar_pfull0, 128);
         mbar_init(bar_pfull0 + 8, 128);
-        mbar_init(bar_odone, 1);
+        mbar_init(bar_odone0, 1);
+        mbar_init(bar_odone0 + 8, 1);
         mbar_init(bar_final, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -486,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_mma_ts(t_o, tp + kk * 8, bdesc, idesc_pv,
                               (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(bar_odone);
+                tc_commit(bar_odone0 + 8 * (j & 1));
                 tc_commit(bar_vempty(s));
                 BD_TRACE(0, (j << 4) | 7);
                 return true;
@@ -575,30 +673,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
                 }
             }
-            float mx = s[0];
+            // row max: 8 independent chains of three-input max
+            float mc[8];
 #pragma unroll
-            for (int c = 1; c < kTcN; ++c)
-                mx = fmaxf(mx, s[c]);
+            for (int i = 0; i < 8; ++i)
+                mc[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+            for (int c = 16; c < kTcN; c += 16)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
+            const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]),
+                                   fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
             const float mt = mx * sl2; // tile max in the log2 domain
-            // PV_{j-1} must be complete before O may be touched and before the
-            // S buffer holding P_{j-1} is reused by the MMA warp
-            if (j >= 1) {
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (j - 1) & 1, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-            }
             // Raise m_used only when the tile max exceeds it by more than 8
             // (in log2 units).  The decision is per row, but the TMEM
             // read-modify-write of O is a warp-collective instruction, so the
             // whole warp takes it when any lane needs it (factor 1 elsewhere).
             const bool need = mt > m_used + 8.f;
+            const bool warp_need = __any_sync(0xffffffffu, need);
             float c = 1.f;
             if (need) {
                 c = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
                 l *= c;
                 m_used = mt;
             }
-            if (j >= 1 && __any_sync(0xffffffffu, need)) {
+            if (j >= 1 && warp_need) {
+                // O is stable once PV_{j-1} has completed (PV_j needs P_j)
+                const int jp = j - 1;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(bar_odone0 + 8 * (jp & 1), (jp >> 1) & 1, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
                 for (int q4 = 0; q4 < kTcD / 32; ++q4) {
                     uint32_t o[32];
@@ -610,29 +716,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tmem_st32(t_o + lane_off + q4 * 32, o);
                 }
             }
-            const float mexp = (m_used == -INFINITY) ? 0.f : m_used;
-            float rs = 0.f;
-#pragma unroll
-            for (int c4 = 0; c4 < kTcN / 32; ++c4) {
-                // P of 32 keys -> 16 packed bf16x2 words over the S columns
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    const float p0 = ex2(fmaf(s[c4 * 32 + c], sl2, -mexp));
-                    const float p1 = ex2(fmaf(s[c4 * 32 + c + 1], sl2, -mexp));
-                    rs += p0 + p1;
-                    pk[c / 2] = pack_bf16x2(p0, p1);
-                }
-                tmem_st16(ts + c4 * 16, pk);
-            }
-            l += rs;
+            const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+            float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+            if (full)
+                softmax_p_tile<kEmuExp2>(s, sl2, nm, ts, rsum);
+            else
+                softmax_p_tile<false>(s, sl2, nm, ts, rsum);
+            l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_pfull0 + 8 * (j & 1));
             if (lane == 0) BD_TRACE(2 + warp, (j << 4) | 3);
         }
         if (ok && nt > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (nt - 1) & 1, abort_flag));
+            const int jl = nt - 1; // PV_{nt-1} done => every PV done
+            ok = __all_sync(0xffffffffu,
+                            mbar_wait(bar_odone0 + 8 * (jl & 1), (jl >> 1) & 1, abort_flag));
             tc_fence_after();
         }
         // epilogue: O / l -> out, lse
