@@ -44,7 +44,7 @@ L2_FLUSH_BYTES = 256 << 20
 # bd_mma_attn_kernel_decode_denoise.md); None whenever the kernel has changed
 # since those counters were taken.
 FWD_TRAFFIC_BYTES = None
-DECODE_TRAFFIC_BYTES = 576815104
+DECODE_TRAFFIC_BYTES = None
 
 
 def fwd_flops(s) -> int:

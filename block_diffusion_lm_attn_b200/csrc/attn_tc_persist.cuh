@@ -1,0 +1,713 @@
+// Persistent tcgen05 block-diffusion attention kernel, shared by the
+// training/prefill form and the block-decode form.
+//
+// The grid is one CTA per SM.  Each CTA walks a list of SEGMENTS; a segment
+// is one 128-row query tile and a run of 128-key K/V tiles:
+//   training/prefill: every (batch, head, query tile) is one segment; the
+//     work items are ordered by cost (key tiles visited) and dealt to the
+//     CTAs in snake order (round k: CTA c takes item k G + c, or
+//     k G + G - 1 - c on odd rounds), which balances the per-CTA totals;
+//   block decode: the (unit, key tile) space -- a unit is one (sequence,
+//     kv-head, 128-row query tile) -- is cut into G equal contiguous ranges
+//     (stream-K).  A unit that lies inside one CTA's range is finished there;
+//     a unit cut by range boundaries leaves a normalised partial (o, lse) per
+//     piece, merged by bd_decode_stream_combine_kernel.
+//
+// Roles (same as the one-tile kernel in attn_tc.cuh): warps 0-3 softmax
+// (thread t = query row t = TMEM lane t), warp 4 TMA producer, warp 5 MMA
+// issuer.  All roles enumerate the same segments in the same order; the
+// K/V ring stage and the S/P/PV barrier phases follow one running tile
+// counter across segments, so the Q load and S = QK^T of the next segment
+// overlap the last PV and the epilogue of the current one.  Q (shared
+// memory) and O (TMEM columns 256-383 and 384-511) are double-buffered by
+// segment parity, with two handshakes per buffer: q_free (every QK of the
+// segment that last used the Q buffer has retired) and o_free (the epilogue
+// that last used the O buffer has read it out).
+#pragma once
+
+#include "attn_tc.cuh"
+
+namespace bd {
+
+struct PParams {
+    bf16 *out;
+    float *lse;
+    float *part_o;   // decode: [G][2][128][128] fp32 partial outputs
+    float *part_lse; // decode: [G][2][128]
+    const int32_t *cache_len;
+    int B, Hq, Hkv, L, b;
+    int nkeys;     // key rows per kv-head: 2L or S_cap
+    int mode;      // decode: 0 bidirectional, 1 causal
+    int qtiles;    // fwd: 128-row query tiles per half
+    int row_tiles; // decode: 128-row query tiles per unit
+    int rows_unit; // decode: query rows per (sequence, kv-head) = group * b
+    int sched_slot; // fwd: counter pair of this launch (0 .. kSchedSlots-1)
+    float scale_log2;
+};
+
+struct Seg {
+    int qhead, qrow0, nrows, kvhead;
+    int lo0, hi0, lo1, hi1;     // key ranges
+    int flo0, fhi0, flo1, fhi1; // keys every row of the tile sees
+    int n0, nt;                 // tiles in range 0, in total
+    int len;            // decode: cache length of the sequence
+    int out_row0;       // decode: global output row of tile row 0
+    int complete;       // decode: the segment covers its whole unit
+    int slot;           // decode: partial slot (0 or 1) of this CTA
+};
+
+// Number of 128-key tiles of one decode unit (0 for an invalid length).
+__device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap)
+{
+    if (len < 0 || (long long)len + b > S_cap)
+        return 0;
+    return (len + b + kTcN - 1) / kTcN;
+}
+
+// ----------------------------------------------------------------------------
+// training / prefill work list
+
+// The work items are handed out dynamically: the TMA producer of each CTA
+// takes the next item index from a global counter and passes it to the MMA
+// and softmax roles through a 4-entry ring in shared memory.  Items are in
+// head-major order, heaviest query tile first inside each (batch, head), so
+// the CTAs running at any moment share the K/V of one or two heads in L2,
+// while the dynamic hand-out keeps their loads balanced.  Each launch uses
+// one of kSchedSlots counter pairs (rotating on the host); the last CTA of a
+// launch to finish resets its pair.
+constexpr int kSchedSlots = 64;
+__device__ unsigned int g_sched_next[kSchedSlots];
+__device__ unsigned int g_sched_done[kSchedSlots];
+
+struct FwdSource {
+    __device__ void init(const PParams &) {}
+    __device__ static long long items(const PParams &p)
+    {
+        return (long long)p.B * p.Hq * 2 * p.qtiles;
+    }
+    // item w: (batch, head) = w / R, cost rank r = w % R (0 = heaviest)
+    __device__ static void item(const PParams &p, int w, Seg &sg)
+    {
+        const int R = 2 * p.qtiles;
+        const int bh = w / R;
+        const int r = w % R;
+        const int idx = p.qtiles - 1 - (r >> 1);
+        const int clean = r & 1; // noisy tile k is one K/V tile heavier
+        sg.qrow0 = (clean ? p.L : 0) + idx * kTcM;
+        sg.nrows = min(kTcM, p.L - idx * kTcM);
+        sg.qhead = bh;
+        sg.kvhead = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
+        const Span first = fwd_span(p.L, p.b, sg.qrow0);
+        const Span last = fwd_span(p.L, p.b, sg.qrow0 + sg.nrows - 1);
+        sg.lo0 = first.a0; sg.hi0 = last.a1;
+        sg.lo1 = first.a2; sg.hi1 = last.a3;
+        sg.flo0 = last.a0; sg.fhi0 = first.a1;
+        sg.flo1 = last.a2; sg.fhi1 = first.a3;
+        sg.n0 = sg.hi0 > sg.lo0 ? (sg.hi0 - sg.lo0 + kTcN - 1) / kTcN : 0;
+        const int n1 = sg.hi1 > sg.lo1 ? (sg.hi1 - sg.lo1 + kTcN - 1) / kTcN : 0;
+        sg.nt = sg.n0 + n1;
+    }
+};
+
+// ----------------------------------------------------------------------------
+// block decode work list (stream-K over units x key tiles)
+
+__device__ __forceinline__ long long range_start(long long T, int G, int c)
+{
+    return T * c / G;
+}
+
+struct DecSource {
+    long long t, t1, t0;  // position, end and start of this CTA's range
+    long long seq_base;   // first global tile of the current sequence
+    int seq, seq_tiles, len;
+
+    __device__ void load_seq(const PParams &p)
+    {
+        len = seq < p.B ? p.cache_len[seq] : 0;
+        seq_tiles = seq < p.B ? decode_unit_tiles(len, p.b, p.nkeys) : 0;
+    }
+    __device__ void init(const PParams &p)
+    {
+        const int ups = p.Hkv * p.row_tiles; // units per sequence
+        long long T = 0;
+        for (int i = 0; i < p.B; ++i)
+            T += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+        t0 = t = range_start(T, gridDim.x, blockIdx.x);
+        t1 = range_start(T, gridDim.x, blockIdx.x + 1);
+        seq = 0;
+        seq_base = 0;
+        load_seq(p);
+    }
+    __device__ bool next(const PParams &p, Seg &sg)
+    {
+        if (t >= t1)
+            return false;
+        const int ups = p.Hkv * p.row_tiles;
+        while (t >= seq_base + (long long)ups * seq_tiles) {
+            seq_base += (long long)ups * seq_tiles;
+            ++seq;
+            load_seq(p);
+        }
+        const long long local = t - seq_base;
+        const int uis = (int)(local / seq_tiles); // unit inside the sequence
+        const int kt0 = (int)(local % seq_tiles);
+        const long long left = t1 - t;
+        const int n = (int)min((long long)(seq_tiles - kt0), left);
+        const int g = uis / p.row_tiles, rt = uis % p.row_tiles;
+        const int group = p.Hq / p.Hkv;
+        sg.qhead = seq * p.Hkv + g;
+        sg.kvhead = sg.qhead;
+        sg.qrow0 = rt * kTcM;
+        sg.nrows = min(kTcM, p.rows_unit - rt * kTcM);
+        sg.lo0 = kt0 * kTcN;
+        sg.hi0 = min((kt0 + n) * kTcN, len + p.b);
+        sg.lo1 = sg.hi1 = 0;
+        sg.flo0 = 0;
+        sg.fhi0 = len + (p.mode == 0 ? p.b : 0);
+        sg.flo1 = sg.fhi1 = 0;
+        sg.n0 = sg.nt = n;
+        sg.len = len;
+        sg.out_row0 = (seq * p.Hq + g * group) * p.b + rt * kTcM;
+        sg.complete = (kt0 == 0 && n == seq_tiles);
+        const long long u0 = seq_base + (long long)uis * seq_tiles;
+        sg.slot = (u0 < t0) ? 0 : 1;
+        t += n;
+        return true;
+    }
+};
+
+// ----------------------------------------------------------------------------
+
+template <int KIND>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    bd_tc_persist_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const PParams p)
+{
+    typedef typename std::conditional<KIND == 0, FwdSource, DecSource>::type Src;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + (base - raw_addr);
+
+    const uint32_t bar0 = base + kSmemBar;
+    const uint32_t bar_q = bar0; // Q buffer 0 landed
+    auto bar_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
+    auto bar_vfull = [&](int s) { return bar0 + 8 * (1 + kTcStages + s); };
+    auto bar_kempty = [&](int s) { return bar0 + 8 * (1 + 2 * kTcStages + s); };
+    auto bar_vempty = [&](int s) { return bar0 + 8 * (1 + 3 * kTcStages + s); };
+    const uint32_t bar_sfull0 = bar0 + 8 * (1 + 4 * kTcStages); // 2
+    const uint32_t bar_pfull0 = bar_sfull0 + 16;                // 2
+    const uint32_t bar_odone0 = bar_pfull0 + 16;                // 2
+    const uint32_t bar_final = bar_odone0 + 16;
+    const uint32_t bar_qfree0 = bar_final + 8; // 2: Q buffer no longer read
+    const uint32_t bar_ofree0 = bar_qfree0 + 16; // 2: O buffer read out
+    const uint32_t bar_qfull1 = bar_ofree0 + 16; // Q buffer 1 landed
+    const uint32_t bar_ifull0 = bar0 + 168;  // 4: work item published
+    const uint32_t bar_iempty0 = bar0 + 200; // 4: work item read by all roles
+    volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kSmemBar + 256);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kSmemBar + 384);
+    volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + kSmemBar + 392);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+            mbar_init(bar_vempty(s), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_sfull0 + 8 * i, 1);
+            mbar_init(bar_pfull0 + 8 * i, 128);
+            mbar_init(bar_odone0 + 8 * i, 1);
+        }
+        mbar_init(bar_final, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_qfree0 + 8 * i, 1);
+            mbar_init(bar_ofree0 + 8 * i, 128);
+        }
+        mbar_init(bar_qfull1, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_ifull0 + 8 * i, 1);
+            mbar_init(bar_iempty0 + 8 * i, 129); // MMA thread + 128 softmax threads
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32((const void *)tmem_slot)), "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s0 = tmem;      // S buffers: columns [0, 128), [128, 256)
+    const uint32_t t_o0 = tmem + 256; // O buffers: columns [256, 384), [384, 512)
+    auto bar_qfull = [&](int i) { return i ? bar_qfull1 : bar_q; };
+
+    Src src;
+    src.init(p);
+    Seg sg;
+
+    // Next segment of this CTA, identical for every role.  Training/prefill:
+    // the producer takes the next item from the global counter and publishes
+    // it in item_ring[si % 4]; the other roles read it there.  Decode: each
+    // role walks its static stream-K range.
+    auto next_seg = [&](int si, bool producer, bool &ok) -> bool {
+        if constexpr (KIND == 1) {
+            return src.next(p, sg);
+        } else {
+        const int slot = si & 3;
+        int w;
+        if (producer) {
+            if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
+                                             (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
+                return false;
+            const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
+            w = (long long)t < FwdSource::items(p) ? (int)t : -1;
+            item_ring[slot] = w;
+            mbar_arrive(bar_ifull0 + 8 * slot);
+        } else {
+            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+                return false;
+            w = item_ring[slot];
+            mbar_arrive(bar_iempty0 + 8 * slot);
+        }
+        if (w < 0)
+            return false;
+        FwdSource::item(p, w, sg);
+        return true;
+        }
+    };
+
+    if (warp == 4) {
+        // ---------------------------------------------------- TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            int si = 0;
+            long long g = 0;   // running K/V tile counter
+            long long kiss = 0, viss = 0;
+            while (ok && next_seg(si, true, ok)) {
+                // Q buffer si & 1 was last read by segment si - 2
+                const int qbuf = si & 1;
+                if (si >= 2 && !(ok = mbar_wait(bar_qfree0 + 8 * qbuf,
+                                                 (uint32_t)(((si - 2) >> 1) & 1), abort_flag)))
+                    break;
+                mbar_expect_tx(bar_qfull(qbuf), kTileBytes);
+                tma_load_3d(base + kSmemQ + qbuf * kTileBytes, &tm_q, 0, sg.qrow0,
+                            sg.qhead, bar_qfull(qbuf));
+                tma_load_3d(base + kSmemQ + qbuf * kTileBytes + kHalfTileBytes, &tm_q,
+                            64, sg.qrow0, sg.qhead, bar_qfull(qbuf));
+                ++si;
+                for (int it = 0; it < sg.nt; ++it, ++g) {
+                    const int ks = it < sg.n0 ? sg.lo0 + it * kTcN
+                                              : sg.lo1 + (it - sg.n0) * kTcN;
+                    const int s = (int)(g % kTcStages);
+                    const uint32_t ph = (uint32_t)((g / kTcStages) & 1) ^ 1u;
+                    if (g >= kTcStages && !(ok = mbar_wait(bar_kempty(s), ph, abort_flag)))
+                        break;
+                    mbar_expect_tx(bar_kfull(s), kTileBytes);
+                    tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks,
+                                sg.kvhead, bar_kfull(s));
+                    tma_load_3d(base + kSmemK + s * kTileBytes + kHalfTileBytes,
+                                &tm_k, 64, ks, sg.kvhead, bar_kfull(s));
+                    kiss = g + 1;
+                    if (g >= kTcStages && !(ok = mbar_wait(bar_vempty(s), ph, abort_flag)))
+                        break;
+                    mbar_expect_tx(bar_vfull(s), kTileBytes);
+                    tma_load_3d(base + kSmemV + s * kTileBytes, &tm_v, 0, ks,
+                                sg.kvhead, bar_vfull(s));
+                    tma_load_3d(base + kSmemV + s * kTileBytes + kHalfTileBytes,
+                                &tm_v, 64, ks, sg.kvhead, bar_vfull(s));
+                    viss = g + 1;
+                }
+            }
+            if (KIND == 0) {
+                // this CTA takes no more items; the last CTA resets the pair
+                __threadfence();
+                if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
+                    g_sched_next[p.sched_slot] = 0;
+                    g_sched_done[p.sched_slot] = 0;
+                    __threadfence();
+                }
+            }
+            // wait (bounded) for every copy this role issued
+            const long long c0 = clock64();
+            auto drain = [&](uint32_t bar, uint32_t par) {
+                while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}
+            };
+            for (int x = si > 2 ? si - 2 : 0; x < si; ++x)
+                drain(bar_qfull(x & 1), (uint32_t)((x >> 1) & 1));
+            for (long long x = kiss > kTcStages ? kiss - kTcStages : 0; x < kiss; ++x)
+                drain(bar_kfull((int)(x % kTcStages)), (uint32_t)((x / kTcStages) & 1));
+            for (long long x = viss > kTcStages ? viss - kTcStages : 0; x < viss; ++x)
+                drain(bar_vfull((int)(x % kTcStages)), (uint32_t)((x / kTcStages) & 1));
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(kTcM, kTcN, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16(kTcM, kTcD, 1);
+            bool ok = true;
+            int si = 0;
+            long long j = 0; // running tile counter
+            auto issue_pv = [&](long long jg, bool first) -> bool {
+                const int s = (int)(jg % kTcStages);
+                // O buffer si & 1 was last read out by segment si - 2
+                if (first && si >= 2 &&
+                    !mbar_wait(bar_ofree0 + 8 * (si & 1), (uint32_t)(((si - 2) >> 1) & 1),
+                               abort_flag))
+                    return false;
+                if (!mbar_wait(bar_pfull0 + 8 * (jg & 1), (uint32_t)((jg >> 1) & 1), abort_flag))
+                    return false;
+                if (!mbar_wait(bar_vfull(s), (uint32_t)((jg / kTcStages) & 1), abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t vb = base + kSmemV + s * kTileBytes;
+                const uint32_t tp = t_s0 + (uint32_t)(jg & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < kTcN / 16; ++kk) {
+                    uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, kHalfTileBytes, 1024);
+                    tc_mma_ts(t_o0 + (uint32_t)(si & 1) * 128, tp + kk * 8, bdesc, idesc_pv,
+                              (!first || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_odone0 + 8 * (jg & 1));
+                tc_commit(bar_vempty(s));
+                return true;
+            };
+            while (ok && next_seg(si, false, ok)) {
+                if (!(ok = mbar_wait(bar_qfull(si & 1), (uint32_t)((si >> 1) & 1), abort_flag)))
+                    break;
+                tc_fence_after();
+                for (int jj = 0; jj < sg.nt && ok; ++jj) {
+                    const long long jg = j + jj;
+                    const int s = (int)(jg % kTcStages);
+                    if (!(ok = mbar_wait(bar_kfull(s), (uint32_t)((jg / kTcStages) & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t kb = base + kSmemK + s * kTileBytes;
+                    const uint32_t qb = base + kSmemQ + (si & 1) * kTileBytes;
+                    const uint32_t ts = t_s0 + (uint32_t)(jg & 1) * 128;
+#pragma unroll
+                    for (int kk = 0; kk < kTcD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                        tc_mma_ss(ts, smem_desc_sw128(qb + off, 16, 1024),
+                                  smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
+                                  kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(bar_sfull0 + 8 * (jg & 1));
+                    tc_commit(bar_kempty(s));
+                    if (jj == sg.nt - 1)
+                        tc_commit(bar_qfree0 + 8 * (si & 1)); // Q buffer no longer read
+                    if (jj >= 1)
+                        ok = issue_pv(jg - 1, jj == 1);
+                }
+                if (ok)
+                    ok = issue_pv(j + sg.nt - 1, sg.nt == 1);
+                j += sg.nt;
+                ++si;
+            }
+            tc_commit(bar_final);
+            const long long c0 = clock64();
+            while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
+        }
+    } else {
+        // ---------------------------------------------------- softmax + epilogue
+        const int row = threadIdx.x;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        long long j = 0;
+        int si = 0;
+        for (;;) {
+            const bool got = next_seg(si, false, ok);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!got || !ok)
+                break;
+            const uint32_t t_o = t_o0 + (uint32_t)(si & 1) * 128; // this segment's O
+            const int rl = min(row, sg.nrows - 1);
+            Span sp;
+            if (KIND == 0) {
+                sp = fwd_span(p.L, p.b, sg.qrow0 + rl);
+            } else {
+                const int jr = (sg.qrow0 + rl) % p.b;
+                sp.a0 = 0;
+                sp.a1 = sg.len + (p.mode == 0 ? p.b : jr + 1);
+                sp.a2 = sp.a3 = 0;
+            }
+            float m_used = -INFINITY, l = 0.f;
+            for (int jj = 0; jj < sg.nt; ++jj) {
+                const long long jg = j + jj;
+                const bool r0 = jj < sg.n0;
+                const int ks = r0 ? sg.lo0 + jj * kTcN : sg.lo1 + (jj - sg.n0) * kTcN;
+                const int khi = r0 ? sg.hi0 : sg.hi1;
+                const int flo = r0 ? sg.flo0 : sg.flo1;
+                const int fhi = r0 ? sg.fhi0 : sg.fhi1;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull0 + 8 * (jg & 1),
+                                                       (uint32_t)((jg >> 1) & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const uint32_t ts = t_s0 + (uint32_t)(jg & 1) * 128 + lane_off;
+                uint32_t sr[128];
+                tmem_ld32(ts + 0, sr + 0);
+                tmem_ld32(ts + 32, sr + 32);
+                tmem_ld32(ts + 64, sr + 64);
+                tmem_ld32(ts + 96, sr + 96);
+                tmem_wait_ld();
+                float s[kTcN];
+#pragma unroll
+                for (int c = 0; c < kTcN; ++c)
+                    s[c] = __uint_as_float(sr[c]);
+                const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
+                if (!full) {
+                    const int e = min(khi, ks + kTcN);
+                    const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
+                    const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
+#pragma unroll
+                    for (int w = 0; w < kTcN / 32; ++w) {
+                        const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                                           range_bits(lo1 - 32 * w, hi1 - 32 * w);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
+                    }
+                }
+                float mc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mc[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+                for (int c = 16; c < kTcN; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
+                const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]),
+                                       fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+                const float mt = mx * sl2;
+                // lazy rescale (threshold 2^8); the TMEM read-modify-write of O
+                // is warp-collective, so the warp takes it if any lane needs it
+                const bool need = mt > m_used + 8.f;
+                const bool warp_need = __any_sync(0xffffffffu, need);
+                float c = 1.f;
+                if (need) {
+                    c = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
+                    l *= c;
+                    m_used = mt;
+                }
+                if (jj >= 1 && warp_need) {
+                    const long long jp = jg - 1; // PV_{jp} done => O stable
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(bar_odone0 + 8 * (jp & 1),
+                                              (uint32_t)((jp >> 1) & 1), abort_flag));
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + lane_off + q4 * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * c);
+                        tmem_st32(t_o + lane_off + q4 * 32, o);
+                    }
+                }
+                const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+                float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+                softmax_p_tile<kEmuExp2>(s, sl2, nm, ts, rsum);
+                l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_pfull0 + 8 * (jg & 1));
+            }
+            if (!ok)
+                break;
+            {
+                const long long jl = j + sg.nt - 1; // last PV of the segment
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_odone0 + 8 * (jl & 1),
+                                                       (uint32_t)((jl >> 1) & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+            }
+            // ------------------------------------------------ epilogue
+            const bool valid = row < sg.nrows;
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+            const bool to_out = (KIND == 0) || sg.complete;
+            size_t grow;
+            if (KIND == 0)
+                grow = (size_t)sg.qhead * 2 * p.L + sg.qrow0 + row;
+            else
+                grow = (size_t)sg.out_row0 + row;
+            const size_t prow = ((size_t)blockIdx.x * 2 + sg.slot) * kTcM + row;
+#pragma unroll
+            for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                uint32_t o[32];
+                tmem_ld32(t_o + lane_off + q4 * 32, o);
+                tmem_wait_ld();
+                if (valid && to_out) {
+                    uint4 *orow = reinterpret_cast<uint4 *>(p.out + grow * kTcD);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+                        v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                        v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+                        v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+                        orow[q4 * 4 + i / 8] = v4;
+                    }
+                } else if (valid) {
+                    float4 *prow4 = reinterpret_cast<float4 *>(p.part_o + prow * kTcD);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        prow4[q4 * 8 + i / 4] = make_float4(
+                            __uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                            __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+                }
+            }
+            if (valid) {
+                if (to_out)
+                    p.lse[grow] = lse_v;
+                else
+                    p.part_lse[prow] = lse_v;
+            }
+            tc_fence_before();
+            mbar_arrive(bar_ofree0 + 8 * (si & 1));
+            j += sg.nt;
+            ++si;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+// Merges the partial results of decode units cut by stream-K range
+// boundaries, and writes NaN rows for sequences with an invalid cache length.
+// One CTA of 128 threads per unit (thread = query row of the unit's tile).
+__global__ void __launch_bounds__(128)
+    bd_decode_stream_combine_kernel(const PParams p, int G)
+{
+    const int unit = blockIdx.x; // (seq * Hkv + g) * row_tiles + rt
+    const int row = threadIdx.x;
+    const int ups = p.Hkv * p.row_tiles;
+    const int seq = unit / ups, uis = unit % ups;
+    const int g = uis / p.row_tiles, rt = uis % p.row_tiles;
+    const int group = p.Hq / p.Hkv;
+    const int nrows = min(kTcM, p.rows_unit - rt * kTcM);
+    const size_t orow = (size_t)(seq * p.Hq + g * group) * p.b + rt * kTcM + row;
+    const int len = p.cache_len[seq];
+    const int tiles = decode_unit_tiles(len, p.b, p.nkeys);
+    if (tiles == 0) {
+        if (row < nrows) {
+            for (int t = 0; t < kTcD; ++t)
+                p.out[orow * kTcD + t] = __float2bfloat16_rn(NAN);
+            p.lse[orow] = NAN;
+        }
+        if (row == 0)
+            raise_device_code(DEV_BAD_CACHE_LEN);
+        return;
+    }
+    // global tile range of this unit: sum of the tiles of earlier sequences
+    __shared__ long long s_part[128];
+    long long acc = 0, T = 0;
+    for (int i = row; i < p.B; i += 128) {
+        const long long ti = (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+        T += ti;
+        if (i < seq)
+            acc += ti;
+    }
+    s_part[row] = acc;
+    __syncthreads();
+    for (int off = 64; off > 0; off >>= 1) {
+        if (row < off)
+            s_part[row] += s_part[row + off];
+        __syncthreads();
+    }
+    const long long before = s_part[0];
+    __syncthreads();
+    s_part[row] = T;
+    __syncthreads();
+    for (int off = 64; off > 0; off >>= 1) {
+        if (row < off)
+            s_part[row] += s_part[row + off];
+        __syncthreads();
+    }
+    T = s_part[0];
+    const long long u0 = before + (long long)uis * tiles;
+    const long long u1 = u0 + tiles;
+    auto cta_of = [&](long long t) {
+        int c = (int)((t * G) / T);
+        while (c + 1 < G && range_start(T, G, c + 1) <= t)
+            ++c;
+        while (c > 0 && range_start(T, G, c) > t)
+            --c;
+        return c;
+    };
+    const int cs = cta_of(u0), ce = cta_of(u1 - 1);
+    if (cs == ce || row >= nrows)
+        return; // finished by one CTA, or a padding row
+    float mx = -INFINITY;
+    for (int c = cs; c <= ce; ++c) {
+        if (range_start(T, G, c) == range_start(T, G, c + 1))
+            continue; // CTA with an empty range holds no piece
+        const int slot = (u0 < range_start(T, G, c)) ? 0 : 1;
+        mx = fmaxf(mx, p.part_lse[((size_t)c * 2 + slot) * kTcM + row]);
+    }
+    float accv[kTcD];
+#pragma unroll
+    for (int t = 0; t < kTcD; ++t)
+        accv[t] = 0.f;
+    float z = 0.f;
+    if (mx != -INFINITY) {
+        for (int c = cs; c <= ce; ++c) {
+            if (range_start(T, G, c) == range_start(T, G, c + 1))
+                continue;
+            const int slot = (u0 < range_start(T, G, c)) ? 0 : 1;
+            const size_t pr = ((size_t)c * 2 + slot) * kTcM + row;
+            const float ls = p.part_lse[pr];
+            if (ls == -INFINITY)
+                continue;
+            const float w = ex2((ls - mx) * kLog2e);
+            z += w;
+            const float4 *src = reinterpret_cast<const float4 *>(p.part_o + pr * kTcD);
+#pragma unroll
+            for (int t = 0; t < kTcD / 4; ++t) {
+                const float4 v = src[t];
+                accv[4 * t] += w * v.x;
+                accv[4 * t + 1] += w * v.y;
+                accv[4 * t + 2] += w * v.z;
+                accv[4 * t + 3] += w * v.w;
+            }
+        }
+    }
+    const float inv = z > 0.f ? 1.f / z : 0.f;
+    uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * kTcD);
+#pragma unroll
+    for (int t = 0; t < kTcD; t += 8) {
+        uint4 v4;
+        v4.x = pack_bf16x2(accv[t] * inv, accv[t + 1] * inv);
+        v4.y = pack_bf16x2(accv[t + 2] * inv, accv[t + 3] * inv);
+        v4.z = pack_bf16x2(accv[t + 4] * inv, accv[t + 5] * inv);
+        v4.w = pack_bf16x2(accv[t + 6] * inv, accv[t + 7] * inv);
+        dst[t / 8] = v4;
+    }
+    p.lse[orow] = z > 0.f ? mx + __logf(z) : -INFINITY;
+}
+
+} // namespace bd

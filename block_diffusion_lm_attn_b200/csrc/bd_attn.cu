@@ -1,11 +1,16 @@
 // C-ABI entry points of libbdattn.so: argument validation, launch planning
 // and kernel launches on the caller's stream.  See include/bd_attn.h for the
 // contract of each call.
+//
+// Kernels: head dim 128 runs on the persistent tcgen05 kernel
+// (attn_tc_persist.cuh) in both forms; head dims 32 and 64 run on the
+// mma.sync kernel (attn_mma.cuh).
 #include "bd_attn.h"
 
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 
 #include <cuda.h>
@@ -13,13 +18,16 @@
 
 #include "attn_mma.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc_persist.cuh"
 #include "bd_common.cuh"
 
 namespace {
 
 using bd::bf16;
 
-constexpr int kNumSMs = 148; // B200; used to size split-KV grids
+// B200 SM count: the persistent grids and the decode workspace are sized
+// for at most this many CTAs.
+constexpr int kMaxGrid = 148;
 
 inline bool aligned16(const void *p)
 {
@@ -30,16 +38,30 @@ inline bool supported_d(int d) { return d == 32 || d == 64 || d == 128; }
 
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
-// Split-KV plan for block decode: keys [0, S_cap) of every (batch, kv-head)
-// are cut into `nsplit` chunks of `chunk` keys (a multiple of 64), enough to
-// give the grid a few CTAs per SM.  A pure function of the sizes, so the
-// workspace query and the launch agree without a device round trip.
+inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int persistent_grid()
+{
+    int dev = 0, sms = kMaxGrid;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ==
+            cudaSuccess &&
+        sms > 0)
+        return sms < kMaxGrid ? sms : kMaxGrid;
+    return kMaxGrid;
+}
+
+// Decode launch plan.  A pure function of the sizes, so the workspace query
+// and the launch agree without a device round trip.
+//   d = 128: stream-K over (unit, key tile) on <= kMaxGrid persistent CTAs;
+//            scratch = 2 partial (o, lse) slots of 128 rows per CTA.
+//   d < 128: split-KV with `nsplit` chunks of `chunk` keys per (sequence,
+//            kv-head, 64-row tile); scratch = nsplit partials per row.
 struct DecodePlan {
+    bool tc;
     int row_tiles, nsplit, chunk;
     size_t rows_all, o_bytes, lse_bytes, total_bytes;
 };
-
-inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
                  DecodePlan &pl)
@@ -48,19 +70,28 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
         Hq % Hkv != 0)
         return false;
     const long long rows = (long long)(Hq / Hkv) * b;
-    pl.row_tiles = (int)cdiv(rows, bd::kMmaBM);
-    const long long units = (long long)B * Hkv * pl.row_tiles;
-    const long long target = 4LL * kNumSMs;
-    long long ns = cdiv(target, units);
-    const long long max_ns = cdiv(S_cap, 256);
-    if (ns > max_ns) ns = max_ns;
-    if (ns < 1) ns = 1;
-    long long chunk = cdiv(cdiv(S_cap, ns), 64) * 64;
-    pl.chunk = (int)chunk;
-    pl.nsplit = (int)cdiv(S_cap, chunk);
     pl.rows_all = (size_t)B * Hq * b;
-    pl.o_bytes = round256((size_t)pl.nsplit * pl.rows_all * d * sizeof(float));
-    pl.lse_bytes = round256((size_t)pl.nsplit * pl.rows_all * sizeof(float));
+    pl.tc = (d == 128);
+    if (pl.tc) {
+        pl.row_tiles = (int)cdiv(rows, bd::kTcM);
+        pl.nsplit = 0;
+        pl.chunk = 0;
+        pl.o_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * bd::kTcD * sizeof(float));
+        pl.lse_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * sizeof(float));
+    } else {
+        pl.row_tiles = (int)cdiv(rows, bd::kMmaBM);
+        const long long units = (long long)B * Hkv * pl.row_tiles;
+        const long long target = 4LL * kMaxGrid;
+        long long ns = cdiv(target, units);
+        const long long max_ns = cdiv(S_cap, 256);
+        if (ns > max_ns) ns = max_ns;
+        if (ns < 1) ns = 1;
+        const long long chunk = cdiv(cdiv(S_cap, ns), 64) * 64;
+        pl.chunk = (int)chunk;
+        pl.nsplit = (int)cdiv(S_cap, chunk);
+        pl.o_bytes = round256((size_t)pl.nsplit * pl.rows_all * d * sizeof(float));
+        pl.lse_bytes = round256((size_t)pl.nsplit * pl.rows_all * sizeof(float));
+    }
     pl.total_bytes = pl.o_bytes + pl.lse_bytes;
     return true;
 }
@@ -140,19 +171,14 @@ bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
     return r == CUDA_SUCCESS;
 }
 
-bd_status launch_fwd_tc(const void *q, const void *k, const void *v,
-                        const bd::TcParams &p, cudaStream_t st)
+template <int KIND>
+bd_status launch_persist(const CUtensorMap &mq, const CUtensorMap &mk,
+                         const CUtensorMap &mv, const bd::PParams &p, int grid,
+                         cudaStream_t st)
 {
-    CUtensorMap mq, mk, mv;
-    const uint64_t N = 2ull * p.L;
-    if (!make_map_rows128(&mq, q, N, (uint64_t)p.B * p.Hq) ||
-        !make_map_rows128(&mk, k, N, (uint64_t)p.B * p.Hkv) ||
-        !make_map_rows128(&mv, v, N, (uint64_t)p.B * p.Hkv))
-        return BD_ERR_CUDA;
-    auto kern = bd::bd_tc_attn_kernel<0>;
+    auto kern = bd::bd_tc_persist_kernel<KIND>;
     if (set_smem(kern, bd::kTcSmemBytes) != BD_OK)
         return BD_ERR_CUDA;
-    dim3 grid(2 * p.qtiles, p.B * p.Hq);
     kern<<<grid, bd::kTcThreads, bd::kTcSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
 }
@@ -184,6 +210,94 @@ bd_status launch_decode_mma(const bd::MmaParams &p, const DecodePlan &pl,
     const int rows_all = p.B * p.Hq * p.b;
     bd::bd_decode_combine_kernel<D><<<(rows_all + 7) / 8, 256, 0, st>>>(p);
     return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+// Host-side checks shared by both decode entry points.
+bd_status decode_validate(const void *q_blk, const void *k_cache,
+                          const void *v_cache, const int32_t *cache_len,
+                          const void *out, const float *lse, int B, int Hq,
+                          int Hkv, int b, int d, int mode, int S_cap,
+                          DecodePlan &pl)
+{
+    if (!q_blk || !k_cache || !v_cache || !cache_len || !out || !lse)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(out) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || S_cap < b)
+        return BD_ERR_INVALID_ARG;
+    if (mode != 0 && mode != 1)
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
+        return BD_ERR_INVALID_ARG;
+    if ((long long)B * Hkv > 65535LL || pl.row_tiles > 65535 ||
+        (long long)B * Hkv * pl.row_tiles > (1LL << 30))
+        return BD_ERR_UNSUPPORTED;
+    return BD_OK;
+}
+
+// Launches block decode with a validated plan and a workspace of at least
+// pl.total_bytes (256-byte aligned).
+bd_status decode_launch(const void *q_blk, const void *k_cache,
+                        const void *v_cache, const int32_t *cache_len,
+                        void *out, float *lse, int B, int Hq, int Hkv, int b,
+                        int d, int mode, cudaStream_t stream, int S_cap,
+                        void *workspace, const DecodePlan &pl)
+{
+    float *part_o = static_cast<float *>(workspace);
+    float *part_lse =
+        reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.o_bytes);
+    const float scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
+    if (pl.tc) {
+        bd::PParams p = {};
+        p.out = static_cast<bf16 *>(out);
+        p.lse = lse;
+        p.part_o = part_o;
+        p.part_lse = part_lse;
+        p.cache_len = cache_len;
+        p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
+        p.nkeys = S_cap;
+        p.mode = mode;
+        p.row_tiles = pl.row_tiles;
+        p.rows_unit = (Hq / Hkv) * b;
+        p.scale_log2 = scale_log2;
+        CUtensorMap mq, mk, mv;
+        if (!make_map_rows128(&mq, q_blk, (uint64_t)p.rows_unit, (uint64_t)B * Hkv) ||
+            !make_map_rows128(&mk, k_cache, (uint64_t)S_cap, (uint64_t)B * Hkv) ||
+            !make_map_rows128(&mv, v_cache, (uint64_t)S_cap, (uint64_t)B * Hkv))
+            return BD_ERR_CUDA;
+        const int G = persistent_grid();
+        bd_status st = launch_persist<1>(mq, mk, mv, p, G, stream);
+        if (st != BD_OK)
+            return st;
+        const int units = B * Hkv * pl.row_tiles;
+        bd::bd_decode_stream_combine_kernel<<<units, 128, 0, stream>>>(p, G);
+        return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+    }
+    bd::MmaParams p = {};
+    p.q = static_cast<const bf16 *>(q_blk);
+    p.k = static_cast<const bf16 *>(k_cache);
+    p.v = static_cast<const bf16 *>(v_cache);
+    p.out = static_cast<bf16 *>(out);
+    p.lse = lse;
+    p.part_o = part_o;
+    p.part_lse = part_lse;
+    p.cache_len = cache_len;
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
+    p.nkeys = S_cap;
+    p.mode = mode;
+    p.chunk = pl.chunk;
+    p.nsplit = pl.nsplit;
+    p.scale_log2 = scale_log2;
+    switch (d) {
+    case 32: return launch_decode_mma<32>(p, pl, stream);
+    default: return launch_decode_mma<64>(p, pl, stream);
+    }
 }
 
 } // namespace
@@ -224,14 +338,26 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
         return BD_ERR_UNSUPPORTED;
 
     if (d == 128) {
-        bd::TcParams tp = {};
-        tp.out = static_cast<bf16 *>(out);
-        tp.lse = lse;
-        tp.B = B; tp.Hq = Hq; tp.Hkv = Hkv; tp.L = L; tp.b = b;
-        tp.nkeys = 2 * L;
-        tp.qtiles = (int)cdiv(L, bd::kTcM);
-        tp.scale_log2 = scale * bd::kLog2e;
-        return launch_fwd_tc(q, k, v, tp, stream);
+        bd::PParams p = {};
+        p.out = static_cast<bf16 *>(out);
+        p.lse = lse;
+        p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
+        p.nkeys = 2 * L;
+        p.qtiles = (int)cdiv(L, bd::kTcM);
+        p.scale_log2 = scale * bd::kLog2e;
+        CUtensorMap mq, mk, mv;
+        const uint64_t N = 2ull * L;
+        if (!make_map_rows128(&mq, q, N, (uint64_t)B * Hq) ||
+            !make_map_rows128(&mk, k, N, (uint64_t)B * Hkv) ||
+            !make_map_rows128(&mv, v, N, (uint64_t)B * Hkv))
+            return BD_ERR_CUDA;
+        static std::atomic<unsigned int> launches{0};
+        p.sched_slot = (int)(launches.fetch_add(1u) % bd::kSchedSlots);
+        const long long items = (long long)B * Hq * 2 * p.qtiles;
+        int G = persistent_grid();
+        if (items < G)
+            G = (int)items;
+        return launch_persist<0>(mq, mk, mv, p, G, stream);
     }
 
     bd::MmaParams p = {};
@@ -265,56 +391,24 @@ bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
                          int d, int intra_block_mode, cudaStream_t stream,
                          int S_cap, void *workspace, size_t workspace_bytes)
 {
-    if (!q_blk || !k_cache || !v_cache || !cache_len || !out || !lse)
-        return BD_ERR_INVALID_ARG;
-    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        !aligned16(out) || !aligned16(lse) ||
-        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
-        return BD_ERR_INVALID_ARG;
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
-        return BD_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0 || S_cap < b)
-        return BD_ERR_INVALID_ARG;
-    if (intra_block_mode != 0 && intra_block_mode != 1)
-        return BD_ERR_INVALID_ARG;
-    if (!supported_d(d))
-        return BD_ERR_UNSUPPORTED;
     DecodePlan pl;
-    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
-        return BD_ERR_INVALID_ARG;
-    if ((long long)B * Hkv > 65535LL || pl.row_tiles > 65535)
-        return BD_ERR_UNSUPPORTED;
+    bd_status st = decode_validate(q_blk, k_cache, v_cache, cache_len, out,
+                                   lse, B, Hq, Hkv, b, d, intra_block_mode,
+                                   S_cap, pl);
+    if (st != BD_OK)
+        return st;
     if (workspace) {
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) ||
             workspace_bytes < pl.total_bytes)
             return BD_ERR_INVALID_ARG;
     } else {
-        bd_status st = get_internal_workspace(pl.total_bytes, &workspace);
+        st = get_internal_workspace(pl.total_bytes, &workspace);
         if (st != BD_OK)
             return st;
     }
-
-    bd::MmaParams p = {};
-    p.q = static_cast<const bf16 *>(q_blk);
-    p.k = static_cast<const bf16 *>(k_cache);
-    p.v = static_cast<const bf16 *>(v_cache);
-    p.out = static_cast<bf16 *>(out);
-    p.lse = lse;
-    p.part_o = static_cast<float *>(workspace);
-    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                           pl.o_bytes);
-    p.cache_len = cache_len;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
-    p.nkeys = S_cap;
-    p.mode = intra_block_mode;
-    p.chunk = pl.chunk;
-    p.nsplit = pl.nsplit;
-    p.scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
-    switch (d) {
-    case 32: return launch_decode_mma<32>(p, pl, stream);
-    case 64: return launch_decode_mma<64>(p, pl, stream);
-    default: return launch_decode_mma<128>(p, pl, stream);
-    }
+    return decode_launch(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq,
+                         Hkv, b, d, intra_block_mode, stream, S_cap, workspace,
+                         pl);
 }
 
 bd_status bd_attn_get_device_status(cudaStream_t stream)
@@ -376,57 +470,25 @@ extern "C" bd_status bd_attn_decode_noalloc(
     const int32_t *cache_len, void *out, float *lse, int B, int Hq, int Hkv,
     int b, int d, int intra_block_mode, cudaStream_t stream, int S_cap)
 {
-    if (!q_blk || !k_cache || !v_cache || !cache_len || !out || !lse)
-        return BD_ERR_INVALID_ARG;
-    if (!aligned16(q_blk) || !aligned16(k_cache) || !aligned16(v_cache) ||
-        !aligned16(out) || !aligned16(lse) ||
-        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
-        return BD_ERR_INVALID_ARG;
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
-        return BD_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0 || S_cap < b)
-        return BD_ERR_INVALID_ARG;
-    if (intra_block_mode != 0 && intra_block_mode != 1)
-        return BD_ERR_INVALID_ARG;
-    if (!supported_d(d))
-        return BD_ERR_UNSUPPORTED;
     DecodePlan pl;
-    if (!decode_plan(B, Hq, Hkv, b, d, S_cap, pl))
-        return BD_ERR_INVALID_ARG;
-    if ((long long)B * Hkv > 65535LL || pl.row_tiles > 65535)
-        return BD_ERR_UNSUPPORTED;
+    bd_status st = decode_validate(q_blk, k_cache, v_cache, cache_len, out,
+                                   lse, B, Hq, Hkv, b, d, intra_block_mode,
+                                   S_cap, pl);
+    if (st != BD_OK)
+        return st;
     if (pl.total_bytes > (size_t)BD_ATTN_NOALLOC_SCRATCH_BYTES)
         return BD_ERR_UNSUPPORTED;
     void *scratch = nullptr;
-    bd_status st = noalloc_scratch_address(&scratch);
+    st = noalloc_scratch_address(&scratch);
     if (st != BD_OK)
         return st;
-
-    bd::MmaParams p = {};
-    p.q = static_cast<const bf16 *>(q_blk);
-    p.k = static_cast<const bf16 *>(k_cache);
-    p.v = static_cast<const bf16 *>(v_cache);
-    p.out = static_cast<bf16 *>(out);
-    p.lse = lse;
-    p.part_o = static_cast<float *>(scratch);
-    p.part_lse = reinterpret_cast<float *>(static_cast<char *>(scratch) +
-                                           pl.o_bytes);
-    p.cache_len = cache_len;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
-    p.nkeys = S_cap;
-    p.mode = intra_block_mode;
-    p.chunk = pl.chunk;
-    p.nsplit = pl.nsplit;
-    p.scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
-    switch (d) {
-    case 32: return launch_decode_mma<32>(p, pl, stream);
-    case 64: return launch_decode_mma<64>(p, pl, stream);
-    default: return launch_decode_mma<128>(p, pl, stream);
-    }
+    return decode_launch(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq,
+                         Hkv, b, d, intra_block_mode, stream, S_cap, scratch,
+                         pl);
 }
 
 #ifdef BD_TC_TRACE
-// Debug builds only: point the tensor-core kernel's progress trace at a
+// Debug builds only: point the tensor-core kernels' progress trace at a
 // host-mapped buffer of 8 words per CTA (NULL disables it).
 extern "C" __attribute__((visibility("default"))) int
 bd_debug_set_trace(void *buf)

@@ -56,7 +56,7 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
         _compare(ref_o, ref_l, out, lse)
 
     # a size whose scratch exceeds the fixed array is refused up front
-    B, Hq, Hkv, b, d, S_cap = 256, 64, 8, 32, 128, 65536
+    B, Hq, Hkv, b, d, S_cap = 256, 64, 8, 32, 64, 65536
     assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) > SCRATCH_MAX
     A = 1 << 20
     st = bd.bd_attn_decode_noalloc(A, A, A, A, A, A, B, Hq, Hkv, b, d, 0,
