@@ -99,6 +99,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase has not completed is suspended
+// in hardware until it completes or about `ns` nanoseconds pass, instead of
+// spinning on the issue slots it shares with the other warps of its SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity), "r"(ns)
+                 : "memory");
+    return ok != 0;
+}
+
+#ifndef BD_WAIT_SLEEP_NS
+#define BD_WAIT_SLEEP_NS 2000
+#endif
+
 // Bounded wait on phase `parity` of barrier `bar`.  Returns false if the
 // CTA was aborted (by this wait running out or by another role).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
@@ -107,17 +128,15 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();
-    for (int it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity))
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, BD_WAIT_SLEEP_NS))
             return true;
-        if ((it & 63) == 63) {
-            if (*abort_flag)
-                return false;
-            if (clock64() - t0 > kWaitCycles) {
-                *abort_flag = 1;
-                raise_device_code(DEV_WAIT_TIMEOUT);
-                return false;
-            }
+        if (*abort_flag)
+            return false;
+        if (clock64() - t0 > kWaitCycles) {
+            *abort_flag = 1;
+            raise_device_code(DEV_WAIT_TIMEOUT);
+            return false;
         }
     }
 }
