@@ -160,13 +160,20 @@ def barrier_sync(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank runs its own replica of the
+    workload, so the job finishes when the slowest one does."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Whole-job rate: all ranks' units over the slowest rank's time (per s)."""
+    return world * units_per_rank / (max_ms * 1e-3)
 
 
 def timed_steps(fn, steps, warmup, flush, world, sampler=None):
@@ -252,7 +259,7 @@ def run_ours(args):
         total_ms = timed_steps(step, args.steps, args.warmup, flush, world,
                                sampler)
         ms = total_ms / args.steps
-        value = world * fwd_flops(s) * args.steps / (total_ms * 1e-3) / 1e12
+        value = job_throughput(fwd_flops(s) * args.steps, world, total_ms) / 1e12
         fwd_kernel_tflops = fwd_flops(s) / (ms * 1e-3) / 1e12
         n_launch = args.steps  # one fwd kernel per step
         rows["fwd_train"] = {"tflops": round(fwd_kernel_tflops, 2),

@@ -97,6 +97,15 @@ def bd_attn_status_string(status):
     return load().bd_attn_status_string(status).decode()
 
 
+def bd_attn_debug_inject_fault(kind):
+    """Test hook (include/bd_attn_debug.h): arm (1) or disarm (0) a one-shot
+    fault that makes a bounded wait of the next head-dim-128 launch run out."""
+    fn = load().bd_attn_debug_inject_fault
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int]
+    return fn(kind)
+
+
 # ---------------------------------------------------------------------------
 # torch-tensor conveniences
 

@@ -76,6 +76,8 @@ __device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap)
 // one of kSchedSlots counter pairs (rotating on the host); the last CTA of a
 // launch to finish resets its pair.
 constexpr int kSchedSlots = 64;
+// one-shot fault injection (see bd_attn_debug.h): CTA 0 skips one K copy
+__device__ int g_fault_skip_k;
 __device__ unsigned int g_sched_next[kSchedSlots];
 __device__ unsigned int g_sched_done[kSchedSlots];
 
@@ -314,6 +316,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t ph = (uint32_t)((g / kTcStages) & 1) ^ 1u;
                     if (g >= kTcStages && !(ok = mbar_wait(bar_kempty(s), ph, abort_flag)))
                         break;
+                    if (g == 0 && blockIdx.x == 0 && atomicExch(&g_fault_skip_k, 0) != 0)
+                        continue; // injected fault: this K tile never arrives
                     mbar_expect_tx(bar_kfull(s), kTileBytes);
                     tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks,
                                 sg.kvhead, bar_kfull(s));

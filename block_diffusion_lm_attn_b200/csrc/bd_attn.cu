@@ -6,6 +6,7 @@
 // (attn_tc_persist.cuh) in both forms; head dims 32 and 64 run on the
 // mma.sync kernel (attn_mma.cuh).
 #include "bd_attn.h"
+#include "bd_attn_debug.h"
 
 #include <cmath>
 #include <cstdint>
@@ -125,12 +126,22 @@ bd_status get_internal_workspace(size_t need, void **out)
     return BD_OK;
 }
 
-template <class K> bd_status set_smem(K kernel, int bytes)
+// Raises the kernel's dynamic shared-memory limit once per device (the
+// attribute is per device; later calls, including ones made while a stream
+// is being captured, skip the runtime call).
+template <auto Kernel> bd_status set_smem(int bytes)
 {
-    // idempotent; cheap enough to repeat per call
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    static std::atomic<unsigned long long> done{0}; // one per kernel
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return BD_ERR_CUDA;
+    const unsigned long long bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit)
+        return BD_OK;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              bytes) != cudaSuccess)
         return BD_ERR_CUDA;
+    done.fetch_or(bit, std::memory_order_acq_rel);
     return BD_OK;
 }
 
@@ -177,7 +188,7 @@ bd_status launch_persist(const CUtensorMap &mq, const CUtensorMap &mk,
                          cudaStream_t st)
 {
     auto kern = bd::bd_tc_persist_kernel<KIND>;
-    if (set_smem(kern, bd::kTcSmemBytes) != BD_OK)
+    if (set_smem<bd::bd_tc_persist_kernel<KIND>>(bd::kTcSmemBytes) != BD_OK)
         return BD_ERR_CUDA;
     kern<<<grid, bd::kTcThreads, bd::kTcSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
@@ -188,7 +199,7 @@ bd_status launch_fwd_mma(const bd::MmaParams &p, cudaStream_t st)
 {
     auto kern = bd::bd_mma_attn_kernel<D, 0>;
     constexpr int smem = bd::mma_smem_bytes<D>();
-    if (set_smem(kern, smem) != BD_OK)
+    if (set_smem<bd::bd_mma_attn_kernel<D, 0>>(smem) != BD_OK)
         return BD_ERR_CUDA;
     dim3 grid(2 * p.qtiles, p.B * p.Hq);
     kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
@@ -201,7 +212,7 @@ bd_status launch_decode_mma(const bd::MmaParams &p, const DecodePlan &pl,
 {
     auto kern = bd::bd_mma_attn_kernel<D, 1>;
     constexpr int smem = bd::mma_smem_bytes<D>();
-    if (set_smem(kern, smem) != BD_OK)
+    if (set_smem<bd::bd_mma_attn_kernel<D, 1>>(smem) != BD_OK)
         return BD_ERR_CUDA;
     dim3 grid(pl.nsplit, pl.row_tiles, p.B * p.Hkv);
     kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
@@ -409,6 +420,15 @@ bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
     return decode_launch(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq,
                          Hkv, b, d, intra_block_mode, stream, S_cap, workspace,
                          pl);
+}
+
+bd_status bd_attn_debug_inject_fault(int kind)
+{
+    if (kind != 0 && kind != 1)
+        return BD_ERR_INVALID_ARG;
+    return cudaMemcpyToSymbol(bd::g_fault_skip_k, &kind, sizeof kind) == cudaSuccess
+               ? BD_OK
+               : BD_ERR_CUDA;
 }
 
 bd_status bd_attn_get_device_status(cudaStream_t stream)

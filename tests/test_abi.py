@@ -109,3 +109,7 @@ def test_product_path_does_not_touch_the_oracle():
             if fn.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 txt = open(os.path.join(dp, fn)).read()
                 assert "oracle" not in txt.lower(), fn
+
+
+def test_fault_hook_rejects_unknown_kind(lib):
+    assert bd.bd_attn_debug_inject_fault(7) == bd.BD_ERR_INVALID_ARG

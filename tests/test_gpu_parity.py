@@ -81,6 +81,9 @@ FWD_GRID = [
     (1, 2, 1, 224, 28, 128),
     (2, 4, 1, 130, 1, 128),
     (1, 16, 2, 384, 4, 128),
+    (1, 1, 1, 64, 8, 128),      # fewer work items than SMs
+    (3, 2, 2, 136, 17, 128),    # ragged query tiles in both halves
+    (1, 4, 1, 512, 512, 128),   # one block per half (b = L)
 ]
 
 
@@ -153,6 +156,10 @@ DEC_GRID = [
     (4, 16, 2, 16, 128, [5, 900, 31, 257], 0),   # 8 heads x 16 rows = 128
     (2, 16, 1, 20, 64, [100, 3000], 1),          # 320 rows: several row tiles
     (1, 2, 2, 64, 128, [700], 0),
+    (1, 8, 1, 40, 128, [5000], 1),       # 320 rows: 3 row tiles, one sequence
+    (1, 2, 1, 200, 128, [300], 1),       # b > 128: rows with no key in a piece
+    (2, 4, 4, 3, 128, [20000, 1], 0),    # one long unit cut across many CTAs
+    (5, 8, 2, 7, 128, [0, 128, 129, 1023, 8000], 1),
 ]
 
 
@@ -213,6 +220,38 @@ def test_decode_matches_fwd_noisy_block():
                         torch.tensor([n], dtype=torch.int32), 0)
     assert (o2.float() - out[:, :, n:n + b].float()).abs().max() <= 2e-2
     assert (l2 - lse[:, :, n:n + b]).abs().max() <= 1e-3
+
+
+def test_decode_is_deterministic_and_graph_capturable():
+    """Same bits on repeated calls; the call captured in a CUDA graph (with
+    an explicit workspace) replays to the same result."""
+    B, Hq, Hkv, b, d = 4, 32, 8, 32, 128
+    lens = [3000, 17, 2048, 511]
+    S_cap = 3100
+    q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
+                                            cache_len=lens, seed=9)
+    q, kc, vc, cl = q.cuda(), kc.cuda(), vc.cuda(), cl.cuda()
+    ws = torch.empty(bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap),
+                     dtype=torch.uint8, device="cuda")
+    o1, l1 = bd.decode(q, kc, vc, cl, 0, workspace=ws)
+    o2, l2 = bd.decode(q, kc, vc, cl, 0, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    out = torch.empty_like(o1)
+    lse = torch.empty_like(l1)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        bd.decode(q, kc, vc, cl, 0, out=out, lse=lse, workspace=ws, stream=s)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            bd.decode(q, kc, vc, cl, 0, out=out, lse=lse, workspace=ws, stream=s)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, o1) and torch.equal(lse, l1)
+    assert bd.device_status() == bd.BD_OK
 
 
 def test_decode_bad_cache_len_is_reported():
