@@ -119,7 +119,20 @@ __device__ __forceinline__ long long range_start(long long T, int G, int c)
     return T * c / G;
 }
 
+// Whole-unit mode: when there are no more units than CTAs and the units are
+// balanced (the longest at most 5/4 of the mean), CTA c streams unit c
+// whole, so no unit is cut and nothing needs merging.  Otherwise the
+// (unit, tile) space is cut into equal stream-K ranges.  Both kernels of a
+// decode launch take this decision from the same device-resident lengths.
+__device__ __forceinline__ bool decode_whole_units(const PParams &p, int G,
+                                                   long long T, int maxt)
+{
+    const long long units = (long long)p.B * p.Hkv * p.row_tiles;
+    return units <= G && (long long)maxt * units * 4 <= T * 5;
+}
+
 struct DecSource {
+    bool whole;           // whole-unit mode (see decode_whole_units)
     long long t, t1, t0;  // position, end and start of this CTA's range
     long long seq_base;   // first global tile of the current sequence
     int seq, seq_tiles, len;
@@ -133,12 +146,29 @@ struct DecSource {
     {
         const int ups = p.Hkv * p.row_tiles; // units per sequence
         long long T = 0;
-        for (int i = 0; i < p.B; ++i)
-            T += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
-        t0 = t = range_start(T, gridDim.x, blockIdx.x);
-        t1 = range_start(T, gridDim.x, blockIdx.x + 1);
+        int maxt = 0;
+        for (int i = 0; i < p.B; ++i) {
+            const int ti = decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+            T += (long long)ups * ti;
+            maxt = max(maxt, ti);
+        }
+        whole = decode_whole_units(p, gridDim.x, T, maxt);
         seq = 0;
         seq_base = 0;
+        if (whole) {
+            // CTA c takes unit c: its global tile range
+            const int u = blockIdx.x;
+            const int us = u / ups;
+            long long base = 0;
+            for (int i = 0; i < p.B && i < us; ++i)
+                base += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+            const int ti = us < p.B ? decode_unit_tiles(p.cache_len[us], p.b, p.nkeys) : 0;
+            t0 = t = base + (long long)(u % ups) * ti;
+            t1 = t + ti;
+        } else {
+            t0 = t = range_start(T, gridDim.x, blockIdx.x);
+            t1 = range_start(T, gridDim.x, blockIdx.x + 1);
+        }
         load_seq(p);
     }
     __device__ bool next(const PParams &p, Seg &sg)
@@ -602,116 +632,157 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 }
 
 // Merges the partial results of decode units cut by stream-K range
-// boundaries, and writes NaN rows for sequences with an invalid cache length.
-// One CTA of 128 threads per unit (thread = query row of the unit's tile).
-__global__ void __launch_bounds__(128)
+// boundaries, and writes NaN rows for sequences with an invalid cache
+// length.  Grid (G, kCombineRowGroups): CTA (c, rg) looks at the unit holding
+// the first tile of range c; if that unit started in range c - 1, its rows
+// rg * 8 .. rg * 8 + 7 are merged here, one warp per row, lane l taking
+// output columns 4l .. 4l + 3 (so every load is independent and coalesced).
+// Every cut unit is thereby merged exactly once, by the boundary just after
+// its first piece; units inside one range were finished by the attention
+// kernel.
+constexpr int kCombineRowGroups = kTcM / 8;
+constexpr int kMaxGridDev = 160; // >= the persistent grid (148 on B200)
+
+__global__ void __launch_bounds__(256)
     bd_decode_stream_combine_kernel(const PParams p, int G)
 {
-    const int unit = blockIdx.x; // (seq * Hkv + g) * row_tiles + rt
-    const int row = threadIdx.x;
-    const int ups = p.Hkv * p.row_tiles;
-    const int seq = unit / ups, uis = unit % ups;
-    const int g = uis / p.row_tiles, rt = uis % p.row_tiles;
+    const int c = blockIdx.x, rg = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ups = p.Hkv * p.row_tiles; // units per sequence
     const int group = p.Hq / p.Hkv;
-    const int nrows = min(kTcM, p.rows_unit - rt * kTcM);
-    const size_t orow = (size_t)(seq * p.Hq + g * group) * p.b + rt * kTcM + row;
-    const int len = p.cache_len[seq];
-    const int tiles = decode_unit_tiles(len, p.b, p.nkeys);
-    if (tiles == 0) {
-        if (row < nrows) {
-            for (int t = 0; t < kTcD; ++t)
-                p.out[orow * kTcD + t] = __float2bfloat16_rn(NAN);
-            p.lse[orow] = NAN;
+
+    if (rg == 0) { // invalid sequences (i % G == c): NaN rows
+        for (int i = c; i < p.B; i += G) {
+            if (decode_unit_tiles(p.cache_len[i], p.b, p.nkeys) != 0)
+                continue;
+            for (int r = threadIdx.x; r < p.Hq * p.b; r += blockDim.x) {
+                const size_t orow = (size_t)i * p.Hq * p.b + r;
+                for (int t = 0; t < kTcD; ++t)
+                    p.out[orow * kTcD + t] = __float2bfloat16_rn(NAN);
+                p.lse[orow] = NAN;
+            }
+            if (threadIdx.x == 0)
+                raise_device_code(DEV_BAD_CACHE_LEN);
         }
-        if (row == 0)
-            raise_device_code(DEV_BAD_CACHE_LEN);
+    }
+    if (c == 0)
         return;
+
+    // warp 0: total tiles T and the unit holding tile tc = start of range c
+    __shared__ long long s_T, s_base;
+    __shared__ int s_seq;
+    if (warp == 0) {
+        const int per = (p.B + 31) / 32;
+        const int i0 = lane * per, i1 = min(p.B, i0 + per);
+        long long part = 0;
+        for (int i = i0; i < i1; ++i)
+            part += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+        long long incl = part;
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o)
+                incl += v;
+        }
+        const long long T = __shfl_sync(0xffffffffu, incl, 31);
+        int maxt = 0;
+        for (int i = i0; i < i1; ++i)
+            maxt = max(maxt, decode_unit_tiles(p.cache_len[i], p.b, p.nkeys));
+        for (int o = 16; o > 0; o >>= 1)
+            maxt = max(maxt, __shfl_xor_sync(0xffffffffu, maxt, o));
+        const long long tc = range_start(T, G, c);
+        const long long excl = incl - part;
+        if (lane == 0) {
+            s_T = T;
+            s_seq = -1; // stays -1 when tc >= T (more CTAs than tiles)
+        }
+        __syncwarp();
+        if (decode_whole_units(p, G, T, maxt)) {
+            // every unit was finished whole by the attention kernel
+        } else
+        if (part > 0 && tc >= excl && tc < incl) {
+            long long base = excl;
+            int i = i0;
+            for (; i < i1; ++i) {
+                const long long ti =
+                    (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+                if (tc < base + ti)
+                    break;
+                base += ti;
+            }
+            s_seq = i;
+            s_base = base;
+        }
     }
-    // global tile range of this unit: sum of the tiles of earlier sequences
-    __shared__ long long s_part[128];
-    long long acc = 0, T = 0;
-    for (int i = row; i < p.B; i += 128) {
-        const long long ti = (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
-        T += ti;
-        if (i < seq)
-            acc += ti;
-    }
-    s_part[row] = acc;
     __syncthreads();
-    for (int off = 64; off > 0; off >>= 1) {
-        if (row < off)
-            s_part[row] += s_part[row + off];
-        __syncthreads();
-    }
-    const long long before = s_part[0];
+    const int seq = s_seq;
+    if (seq < 0)
+        return;
+    const long long T = s_T;
+    // range starts of all CTAs, one 64-bit division per thread at most
+    __shared__ long long s_rs[kMaxGridDev + 1];
+    for (int x = threadIdx.x; x <= G; x += blockDim.x)
+        s_rs[x] = range_start(T, G, x);
     __syncthreads();
-    s_part[row] = T;
-    __syncthreads();
-    for (int off = 64; off > 0; off >>= 1) {
-        if (row < off)
-            s_part[row] += s_part[row + off];
-        __syncthreads();
-    }
-    T = s_part[0];
-    const long long u0 = before + (long long)uis * tiles;
-    const long long u1 = u0 + tiles;
-    auto cta_of = [&](long long t) {
-        int c = (int)((t * G) / T);
-        while (c + 1 < G && range_start(T, G, c + 1) <= t)
-            ++c;
-        while (c > 0 && range_start(T, G, c) > t)
-            --c;
-        return c;
+    const long long tc = s_rs[c];
+    const int tiles = decode_unit_tiles(p.cache_len[seq], p.b, p.nkeys);
+    const int uis = (int)((tc - s_base) / tiles);
+    const long long u0 = s_base + (long long)uis * tiles;
+    if (u0 == tc)
+        return; // the unit starts exactly at this boundary: not cut here
+    auto cta_of = [&](long long t) { // x with s_rs[x] <= t < s_rs[x + 1]
+        int lo = 0, hi = G; // invariant: s_rs[lo] <= t < s_rs[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_rs[mid] <= t)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        return lo;
     };
-    const int cs = cta_of(u0), ce = cta_of(u1 - 1);
-    if (cs == ce || row >= nrows)
-        return; // finished by one CTA, or a padding row
+    const int cs = cta_of(u0);
+    if (cs != c - 1)
+        return; // the unit was cut earlier: merged by that boundary's CTAs
+    const int ce = cta_of(u0 + tiles - 1);
+    const int g = uis / p.row_tiles, rt = uis % p.row_tiles;
+    const int nrows = min(kTcM, p.rows_unit - rt * kTcM);
+    const int r = rg * 8 + warp;
+    if (r >= nrows)
+        return;
+    const size_t orow = (size_t)(seq * p.Hq + g * group) * p.b + rt * kTcM + r;
     float mx = -INFINITY;
-    for (int c = cs; c <= ce; ++c) {
-        if (range_start(T, G, c) == range_start(T, G, c + 1))
+    for (int x = cs; x <= ce; ++x) {
+        const long long a = s_rs[x];
+        if (a == s_rs[x + 1])
             continue; // CTA with an empty range holds no piece
-        const int slot = (u0 < range_start(T, G, c)) ? 0 : 1;
-        mx = fmaxf(mx, p.part_lse[((size_t)c * 2 + slot) * kTcM + row]);
+        const size_t pr = ((size_t)x * 2 + (u0 < a ? 0 : 1)) * kTcM + r;
+        mx = fmaxf(mx, p.part_lse[pr]);
     }
-    float accv[kTcD];
-#pragma unroll
-    for (int t = 0; t < kTcD; ++t)
-        accv[t] = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     float z = 0.f;
     if (mx != -INFINITY) {
-        for (int c = cs; c <= ce; ++c) {
-            if (range_start(T, G, c) == range_start(T, G, c + 1))
+        for (int x = cs; x <= ce; ++x) {
+            const long long a = s_rs[x];
+            if (a == s_rs[x + 1])
                 continue;
-            const int slot = (u0 < range_start(T, G, c)) ? 0 : 1;
-            const size_t pr = ((size_t)c * 2 + slot) * kTcM + row;
+            const size_t pr = ((size_t)x * 2 + (u0 < a ? 0 : 1)) * kTcM + r;
             const float ls = p.part_lse[pr];
-            if (ls == -INFINITY)
-                continue;
-            const float w = ex2((ls - mx) * kLog2e);
+            const float4 v = reinterpret_cast<const float4 *>(p.part_o + pr * kTcD)[lane];
+            const float w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
             z += w;
-            const float4 *src = reinterpret_cast<const float4 *>(p.part_o + pr * kTcD);
-#pragma unroll
-            for (int t = 0; t < kTcD / 4; ++t) {
-                const float4 v = src[t];
-                accv[4 * t] += w * v.x;
-                accv[4 * t + 1] += w * v.y;
-                accv[4 * t + 2] += w * v.z;
-                accv[4 * t + 3] += w * v.w;
-            }
+            acc.x += w * v.x;
+            acc.y += w * v.y;
+            acc.z += w * v.z;
+            acc.w += w * v.w;
         }
     }
     const float inv = z > 0.f ? 1.f / z : 0.f;
-    uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * kTcD);
-#pragma unroll
-    for (int t = 0; t < kTcD; t += 8) {
-        uint4 v4;
-        v4.x = pack_bf16x2(accv[t] * inv, accv[t + 1] * inv);
-        v4.y = pack_bf16x2(accv[t + 2] * inv, accv[t + 3] * inv);
-        v4.z = pack_bf16x2(accv[t + 4] * inv, accv[t + 5] * inv);
-        v4.w = pack_bf16x2(accv[t + 6] * inv, accv[t + 7] * inv);
-        dst[t / 8] = v4;
-    }
-    p.lse[orow] = z > 0.f ? mx + __logf(z) : -INFINITY;
+    uint2 o2;
+    o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    reinterpret_cast<uint2 *>(p.out + orow * kTcD)[lane] = o2;
+    if (lane == 0)
+        p.lse[orow] = z > 0.f ? mx + __logf(z) : -INFINITY;
 }
 
 } // namespace bd

@@ -286,8 +286,8 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
         bd_status st = launch_persist<1>(mq, mk, mv, p, G, stream);
         if (st != BD_OK)
             return st;
-        const int units = B * Hkv * pl.row_tiles;
-        bd::bd_decode_stream_combine_kernel<<<units, 128, 0, stream>>>(p, G);
+        bd::bd_decode_stream_combine_kernel<<<dim3(G, bd::kCombineRowGroups), 256, 0,
+                                              stream>>>(p, G);
         return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
     }
     bd::MmaParams p = {};
