@@ -327,6 +327,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             int si = 0;
             long long g = 0;   // running K/V tile counter
             long long kiss = 0, viss = 0;
+            // Decode: V of a tile is issued after K of the next one, so the
+            // K load that QK waits for never queues behind a V load (PV
+            // needs V a whole softmax later); measured ~3% faster there.
+            // Forward: V follows its own K at once (deferring it measured
+            // ~1% slower on long sequences).  pv_*: the V load not issued.
+            bool pv = false, pv_skip = false;
+            int pv_ks = 0, pv_head = 0;
+            long long pv_g = 0;
+            auto issue_v = [&]() -> bool {
+                const int s = (int)(pv_g % kTcStages);
+                const uint32_t ph = (uint32_t)((pv_g / kTcStages) & 1) ^ 1u;
+                pv = false;
+                if (pv_skip)
+                    return true;
+                if (pv_g >= kTcStages && !mbar_wait(bar_vempty(s), ph, abort_flag))
+                    return false;
+                mbar_expect_tx(bar_vfull(s), kTileBytes);
+                tma_load_3d(base + kSmemV + s * kTileBytes, &tm_v, 0, pv_ks, pv_head,
+                            bar_vfull(s));
+                tma_load_3d(base + kSmemV + s * kTileBytes + kHalfTileBytes, &tm_v, 64,
+                            pv_ks, pv_head, bar_vfull(s));
+                viss = pv_g + 1;
+                return true;
+            };
             while (ok && next_seg(si, true, ok)) {
                 // Q buffer si & 1 was last read by segment si - 2
                 const int qbuf = si & 1;
@@ -346,24 +370,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t ph = (uint32_t)((g / kTcStages) & 1) ^ 1u;
                     if (g >= kTcStages && !(ok = mbar_wait(bar_kempty(s), ph, abort_flag)))
                         break;
+                    bool skip = false;
                     if (g == 0 && blockIdx.x == 0 && atomicExch(&g_fault_skip_k, 0) != 0)
-                        continue; // injected fault: this K tile never arrives
-                    mbar_expect_tx(bar_kfull(s), kTileBytes);
-                    tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks,
-                                sg.kvhead, bar_kfull(s));
-                    tma_load_3d(base + kSmemK + s * kTileBytes + kHalfTileBytes,
-                                &tm_k, 64, ks, sg.kvhead, bar_kfull(s));
-                    kiss = g + 1;
-                    if (g >= kTcStages && !(ok = mbar_wait(bar_vempty(s), ph, abort_flag)))
+                        skip = true; // injected fault: this tile never arrives
+                    if (!skip) {
+                        mbar_expect_tx(bar_kfull(s), kTileBytes);
+                        tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks,
+                                    sg.kvhead, bar_kfull(s));
+                        tma_load_3d(base + kSmemK + s * kTileBytes + kHalfTileBytes,
+                                    &tm_k, 64, ks, sg.kvhead, bar_kfull(s));
+                        kiss = g + 1;
+                    }
+                    if (pv && !(ok = issue_v()))
                         break;
-                    mbar_expect_tx(bar_vfull(s), kTileBytes);
-                    tma_load_3d(base + kSmemV + s * kTileBytes, &tm_v, 0, ks,
-                                sg.kvhead, bar_vfull(s));
-                    tma_load_3d(base + kSmemV + s * kTileBytes + kHalfTileBytes,
-                                &tm_v, 64, ks, sg.kvhead, bar_vfull(s));
-                    viss = g + 1;
+                    pv = true;
+                    pv_skip = skip;
+                    pv_ks = ks;
+                    pv_head = sg.kvhead;
+                    pv_g = g;
+                    if (KIND == 0 && !(ok = issue_v()))
+                        break;
                 }
             }
+            if (ok && pv)
+                ok = issue_v();
             if (KIND == 0) {
                 // this CTA takes no more items; the last CTA resets the pair
                 __threadfence();
