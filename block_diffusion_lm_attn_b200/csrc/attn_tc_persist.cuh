@@ -34,6 +34,8 @@ struct PParams {
     float *lse;
     float *part_o;   // decode: [G][2][128][128] fp32 partial outputs
     float *part_lse; // decode: [G][2][128]
+    int4 *cut_desc;  // decode: [G] unit cut at the end of CTA c's range:
+                     // {rows (0: none), CTA of its last tile, out row, 0}
     const int32_t *cache_len;
     int B, Hq, Hkv, L, b;
     int nkeys;     // key rows per kv-head: 2L or S_cap
@@ -54,6 +56,8 @@ struct Seg {
     int out_row0;       // decode: global output row of tile row 0
     int complete;       // decode: the segment covers its whole unit
     int slot;           // decode: partial slot (0 or 1) of this CTA
+    int last_cta;       // decode: CTA holding the unit's last tile (cut
+                        // units that start in this CTA's range), else -1
 };
 
 // Number of 128-key tiles of one decode unit (0 for an invalid length).
@@ -134,6 +138,7 @@ __device__ __forceinline__ bool decode_whole_units(const PParams &p, int G,
 struct DecSource {
     bool whole;           // whole-unit mode (see decode_whole_units)
     long long t, t1, t0;  // position, end and start of this CTA's range
+    long long T;          // tiles of the whole launch
     long long seq_base;   // first global tile of the current sequence
     int seq, seq_tiles, len;
 
@@ -145,7 +150,7 @@ struct DecSource {
     __device__ void init(const PParams &p)
     {
         const int ups = p.Hkv * p.row_tiles; // units per sequence
-        long long T = 0;
+        T = 0;
         int maxt = 0;
         for (int i = 0; i < p.B; ++i) {
             const int ti = decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
@@ -204,6 +209,11 @@ struct DecSource {
         sg.complete = (kt0 == 0 && n == seq_tiles);
         const long long u0 = seq_base + (long long)uis * seq_tiles;
         sg.slot = (u0 < t0) ? 0 : 1;
+        // range x starts at floor(T x / G), so the last x starting at or
+        // before tile e is floor(((e + 1) G - 1) / T)
+        sg.last_cta = (!sg.complete && sg.slot == 1)
+                          ? (int)(((u0 + seq_tiles) * gridDim.x - 1) / T)
+                          : -1;
         t += n;
         return true;
     }
@@ -288,6 +298,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     Src src;
     src.init(p);
     Seg sg;
+    if constexpr (KIND == 1) {
+        // the combine kernel may be scheduled now; it reads nothing of this
+        // launch before the whole grid has finished
+        asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+        if (threadIdx.x == 0)
+            p.cut_desc[blockIdx.x] = make_int4(0, 0, 0, 0);
+        // an empty range (more CTAs than tiles) contributes an empty piece
+        // to any cut unit that spans it
+        if (src.t0 == src.t1 && threadIdx.x < kTcM)
+            p.part_lse[(size_t)blockIdx.x * 2 * kTcM + threadIdx.x] = -INFINITY;
+    }
 
     // Next segment of this CTA, identical for every role.  Training/prefill:
     // the producer takes the next item from the global counter and publishes
@@ -646,6 +667,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 else
                     p.part_lse[prow] = lse_v;
             }
+            if (KIND == 1 && !to_out && sg.last_cta >= 0 && row == 0)
+                p.cut_desc[blockIdx.x] = make_int4(sg.nrows, sg.last_cta, sg.out_row0, 0);
             tc_fence_before();
             mbar_arrive(bar_ofree0 + 8 * (si & 1));
             j += sg.nt;
@@ -663,26 +686,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // Merges the partial results of decode units cut by stream-K range
 // boundaries, and writes NaN rows for sequences with an invalid cache
-// length.  Grid (G, kCombineRowGroups): CTA (c, rg) looks at the unit holding
-// the first tile of range c; if that unit started in range c - 1, its rows
-// rg * 8 .. rg * 8 + 7 are merged here, one warp per row, lane l taking
-// output columns 4l .. 4l + 3 (so every load is independent and coalesced).
-// Every cut unit is thereby merged exactly once, by the boundary just after
-// its first piece; units inside one range were finished by the attention
-// kernel.
-constexpr int kCombineRowGroups = kTcM / 8;
-constexpr int kMaxGridDev = 160; // >= the persistent grid (148 on B200)
+// length.  The attention kernel leaves, for every CTA c whose range ends
+// inside a unit that started in it, a descriptor: the unit's rows, its output
+// row and the CTA x_e holding its last tile.  The unit's pieces are slot 1 of
+// CTA c and slot 0 of CTAs c + 1 .. x_e (an empty range holds an empty
+// piece).  Grid (G, kCombineRowGroups): CTA (c, rg) merges rows
+// rg * 32 .. rg * 32 + 31 of the unit of descriptor c, warp w taking four
+// rows and lane l output columns 4l .. 4l + 3, so every load is coalesced and
+// the four rows' loads are independent.  Launched as a programmatic
+// dependent of the attention kernel: it may start while that kernel runs,
+// and waits for it to finish before reading anything it wrote.
+constexpr int kCombineRowsPerWarp = 4;
+constexpr int kCombineRowGroups = kTcM / (8 * kCombineRowsPerWarp);
 
 __global__ void __launch_bounds__(256)
-    bd_decode_stream_combine_kernel(const PParams p, int G)
+    bd_decode_stream_combine_kernel(const PParams p)
 {
     const int c = blockIdx.x, rg = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ups = p.Hkv * p.row_tiles; // units per sequence
-    const int group = p.Hq / p.Hkv;
+    constexpr int R = kCombineRowsPerWarp;
 
-    if (rg == 0) { // invalid sequences (i % G == c): NaN rows
-        for (int i = c; i < p.B; i += G) {
+    if (rg == 0) { // invalid sequences (i % G == c): NaN rows; the
+                   // attention kernel writes nothing for them
+        for (int i = c; i < p.B; i += gridDim.x) {
             if (decode_unit_tiles(p.cache_len[i], p.b, p.nkeys) != 0)
                 continue;
             for (int r = threadIdx.x; r < p.Hq * p.b; r += blockDim.x) {
@@ -695,124 +721,57 @@ __global__ void __launch_bounds__(256)
                 raise_device_code(DEV_BAD_CACHE_LEN);
         }
     }
-    if (c == 0)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int4 desc = p.cut_desc[c];
+    const int nrows = desc.x, last = desc.y;
+    const int r0 = (rg * 8 + warp) * R;
+    if (r0 >= nrows)
         return;
-
-    // warp 0: total tiles T and the unit holding tile tc = start of range c
-    __shared__ long long s_T, s_base;
-    __shared__ int s_seq;
-    if (warp == 0) {
-        const int per = (p.B + 31) / 32;
-        const int i0 = lane * per, i1 = min(p.B, i0 + per);
-        long long part = 0;
-        for (int i = i0; i < i1; ++i)
-            part += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
-        long long incl = part;
-        for (int o = 1; o < 32; o <<= 1) {
-            const long long v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o)
-                incl += v;
+    float m[R], z[R];
+    float4 acc[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        m[k] = -INFINITY;
+        z[k] = 0.f;
+        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int x = c; x <= last; ++x) {
+        const size_t pr0 = ((size_t)x * 2 + (x == c ? 1 : 0)) * kTcM + r0;
+        float ls[R];
+        float4 v[R];
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            ls[k] = p.part_lse[pr0 + k];
+            v[k] = reinterpret_cast<const float4 *>(p.part_o + (pr0 + k) * kTcD)[lane];
         }
-        const long long T = __shfl_sync(0xffffffffu, incl, 31);
-        int maxt = 0;
-        for (int i = i0; i < i1; ++i)
-            maxt = max(maxt, decode_unit_tiles(p.cache_len[i], p.b, p.nkeys));
-        for (int o = 16; o > 0; o >>= 1)
-            maxt = max(maxt, __shfl_xor_sync(0xffffffffu, maxt, o));
-        const long long tc = range_start(T, G, c);
-        const long long excl = incl - part;
-        if (lane == 0) {
-            s_T = T;
-            s_seq = -1; // stays -1 when tc >= T (more CTAs than tiles)
-        }
-        __syncwarp();
-        if (decode_whole_units(p, G, T, maxt)) {
-            // every unit was finished whole by the attention kernel
-        } else
-        if (part > 0 && tc >= excl && tc < incl) {
-            long long base = excl;
-            int i = i0;
-            for (; i < i1; ++i) {
-                const long long ti =
-                    (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
-                if (tc < base + ti)
-                    break;
-                base += ti;
-            }
-            s_seq = i;
-            s_base = base;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            if (r0 + k >= nrows || ls[k] == -INFINITY)
+                continue; // no row here, or no visible key in this piece
+            const float mn = fmaxf(m[k], ls[k]);
+            const float a = ex2((m[k] - mn) * kLog2e); // 0 while m is -inf
+            const float w = ex2((ls[k] - mn) * kLog2e);
+            z[k] = z[k] * a + w;
+            acc[k].x = acc[k].x * a + w * v[k].x;
+            acc[k].y = acc[k].y * a + w * v[k].y;
+            acc[k].z = acc[k].z * a + w * v[k].z;
+            acc[k].w = acc[k].w * a + w * v[k].w;
+            m[k] = mn;
         }
     }
-    __syncthreads();
-    const int seq = s_seq;
-    if (seq < 0)
-        return;
-    const long long T = s_T;
-    // range starts of all CTAs, one 64-bit division per thread at most
-    __shared__ long long s_rs[kMaxGridDev + 1];
-    for (int x = threadIdx.x; x <= G; x += blockDim.x)
-        s_rs[x] = range_start(T, G, x);
-    __syncthreads();
-    const long long tc = s_rs[c];
-    const int tiles = decode_unit_tiles(p.cache_len[seq], p.b, p.nkeys);
-    const int uis = (int)((tc - s_base) / tiles);
-    const long long u0 = s_base + (long long)uis * tiles;
-    if (u0 == tc)
-        return; // the unit starts exactly at this boundary: not cut here
-    auto cta_of = [&](long long t) { // x with s_rs[x] <= t < s_rs[x + 1]
-        int lo = 0, hi = G; // invariant: s_rs[lo] <= t < s_rs[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (s_rs[mid] <= t)
-                lo = mid;
-            else
-                hi = mid;
-        }
-        return lo;
-    };
-    const int cs = cta_of(u0);
-    if (cs != c - 1)
-        return; // the unit was cut earlier: merged by that boundary's CTAs
-    const int ce = cta_of(u0 + tiles - 1);
-    const int g = uis / p.row_tiles, rt = uis % p.row_tiles;
-    const int nrows = min(kTcM, p.rows_unit - rt * kTcM);
-    const int r = rg * 8 + warp;
-    if (r >= nrows)
-        return;
-    const size_t orow = (size_t)(seq * p.Hq + g * group) * p.b + rt * kTcM + r;
-    float mx = -INFINITY;
-    for (int x = cs; x <= ce; ++x) {
-        const long long a = s_rs[x];
-        if (a == s_rs[x + 1])
-            continue; // CTA with an empty range holds no piece
-        const size_t pr = ((size_t)x * 2 + (u0 < a ? 0 : 1)) * kTcM + r;
-        mx = fmaxf(mx, p.part_lse[pr]);
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+        if (r0 + k >= nrows)
+            break;
+        const size_t orow = (size_t)desc.z + r0 + k;
+        const float inv = z[k] > 0.f ? 1.f / z[k] : 0.f;
+        uint2 o2;
+        o2.x = pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
+        o2.y = pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
+        reinterpret_cast<uint2 *>(p.out + orow * kTcD)[lane] = o2;
+        if (lane == 0)
+            p.lse[orow] = z[k] > 0.f ? m[k] + __logf(z[k]) : -INFINITY;
     }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float z = 0.f;
-    if (mx != -INFINITY) {
-        for (int x = cs; x <= ce; ++x) {
-            const long long a = s_rs[x];
-            if (a == s_rs[x + 1])
-                continue;
-            const size_t pr = ((size_t)x * 2 + (u0 < a ? 0 : 1)) * kTcM + r;
-            const float ls = p.part_lse[pr];
-            const float4 v = reinterpret_cast<const float4 *>(p.part_o + pr * kTcD)[lane];
-            const float w = (ls == -INFINITY) ? 0.f : ex2((ls - mx) * kLog2e);
-            z += w;
-            acc.x += w * v.x;
-            acc.y += w * v.y;
-            acc.z += w * v.z;
-            acc.w += w * v.w;
-        }
-    }
-    const float inv = z > 0.f ? 1.f / z : 0.f;
-    uint2 o2;
-    o2.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    o2.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    reinterpret_cast<uint2 *>(p.out + orow * kTcD)[lane] = o2;
-    if (lane == 0)
-        p.lse[orow] = z > 0.f ? mx + __logf(z) : -INFINITY;
 }
 
 } // namespace bd

@@ -61,7 +61,7 @@ int persistent_grid()
 struct DecodePlan {
     bool tc;
     int row_tiles, nsplit, chunk;
-    size_t rows_all, o_bytes, lse_bytes, total_bytes;
+    size_t rows_all, o_bytes, lse_bytes, desc_bytes, total_bytes;
 };
 
 bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
@@ -79,6 +79,7 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
         pl.chunk = 0;
         pl.o_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * bd::kTcD * sizeof(float));
         pl.lse_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * sizeof(float));
+        pl.desc_bytes = round256((size_t)kMaxGrid * sizeof(int4));
     } else {
         pl.row_tiles = (int)cdiv(rows, bd::kMmaBM);
         const long long units = (long long)B * Hkv * pl.row_tiles;
@@ -92,8 +93,9 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
         pl.nsplit = (int)cdiv(S_cap, chunk);
         pl.o_bytes = round256((size_t)pl.nsplit * pl.rows_all * d * sizeof(float));
         pl.lse_bytes = round256((size_t)pl.nsplit * pl.rows_all * sizeof(float));
+        pl.desc_bytes = 0;
     }
-    pl.total_bytes = pl.o_bytes + pl.lse_bytes;
+    pl.total_bytes = pl.o_bytes + pl.lse_bytes + pl.desc_bytes;
     return true;
 }
 
@@ -270,6 +272,8 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
         p.lse = lse;
         p.part_o = part_o;
         p.part_lse = part_lse;
+        p.cut_desc = reinterpret_cast<int4 *>(static_cast<char *>(workspace) + pl.o_bytes +
+                                              pl.lse_bytes);
         p.cache_len = cache_len;
         p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
         p.nkeys = S_cap;
@@ -286,8 +290,20 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
         bd_status st = launch_persist<1>(mq, mk, mv, p, G, stream);
         if (st != BD_OK)
             return st;
-        bd::bd_decode_stream_combine_kernel<<<dim3(G, bd::kCombineRowGroups), 256, 0,
-                                              stream>>>(p, G);
+        // programmatic dependent launch: the combine's blocks may be placed
+        // while the attention kernel runs; they wait for its end in-kernel
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(G, bd::kCombineRowGroups);
+        cfg.blockDim = dim3(256);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, bd::bd_decode_stream_combine_kernel, p) != cudaSuccess)
+            return BD_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
     }
     bd::MmaParams p = {};
