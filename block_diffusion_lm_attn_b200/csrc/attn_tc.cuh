@@ -26,7 +26,7 @@
 
 namespace bd {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 224; // 4 softmax warps, K producer, MMA, V producer
 constexpr int kTcM = 128;     // query rows per CTA
 constexpr int kTcN = 128;     // keys per K/V tile
 constexpr int kTcD = 128;     // head dim
@@ -34,6 +34,9 @@ constexpr int kTcD = 128;     // head dim
 #define BD_TC_STAGES 2
 #endif
 constexpr int kTcStages = BD_TC_STAGES; // K/V ring depth
+// TMEM S/P buffers of the persistent kernel (128 columns each; O takes the
+// remaining 128 of the 512)
+constexpr int kSBufs = 3;
 #ifndef BD_EXP2_EMU
 #define BD_EXP2_EMU 1
 #endif

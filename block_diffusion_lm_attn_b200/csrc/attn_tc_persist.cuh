@@ -3,26 +3,28 @@
 //
 // The grid is one CTA per SM.  Each CTA walks a list of SEGMENTS; a segment
 // is one 128-row query tile and a run of 128-key K/V tiles:
-//   training/prefill: every (batch, head, query tile) is one segment; the
-//     work items are ordered by cost (key tiles visited) and dealt to the
-//     CTAs in snake order (round k: CTA c takes item k G + c, or
-//     k G + G - 1 - c on odd rounds), which balances the per-CTA totals;
+//   training/prefill: every (batch, head, query tile) is one work item,
+//     handed out dynamically from a global counter (heaviest first inside
+//     each head, see FwdSource);
 //   block decode: the (unit, key tile) space -- a unit is one (sequence,
 //     kv-head, 128-row query tile) -- is cut into G equal contiguous ranges
-//     (stream-K).  A unit that lies inside one CTA's range is finished there;
-//     a unit cut by range boundaries leaves a normalised partial (o, lse) per
+//     (stream-K), or, when the units are few and balanced, dealt one unit
+//     per CTA.  A unit that lies inside one CTA's range is finished there; a
+//     unit cut by range boundaries leaves a normalised partial (o, lse) per
 //     piece, merged by bd_decode_stream_combine_kernel.
 //
-// Roles (same as the one-tile kernel in attn_tc.cuh): warps 0-3 softmax
-// (thread t = query row t = TMEM lane t), warp 4 TMA producer, warp 5 MMA
-// issuer.  All roles enumerate the same segments in the same order; the
-// K/V ring stage and the S/P/PV barrier phases follow one running tile
-// counter across segments, so the Q load and S = QK^T of the next segment
-// overlap the last PV and the epilogue of the current one.  Q (shared
-// memory) and O (TMEM columns 256-383 and 384-511) are double-buffered by
-// segment parity, with two handshakes per buffer: q_free (every QK of the
-// segment that last used the Q buffer has retired) and o_free (the epilogue
-// that last used the O buffer has read it out).
+// Roles: warps 0-3 softmax and epilogue (thread t = query row t = TMEM lane
+// t), warp 4 TMA producer of Q and K, warp 5 MMA issuer, warp 6 TMA producer
+// of V.  All roles enumerate the same segments in the same order; the K/V
+// ring stage and the S/P/PV barrier phases follow one running tile counter
+// across segments, so the Q load and S = QK^T of the next segment overlap
+// the last PV and the epilogue of the current one.  TMEM holds kSBufs = 3
+// S/P buffers (P, bf16, overwrites its own S) and one O; the forward issues
+// QK two tiles ahead of PV, so the softmax warps find the next S ready.  Q
+// is double-buffered in shared memory by segment parity (q_free: every QK of
+// the segment that last used the buffer has retired); O is read out by the
+// epilogue before the softmax of the next segment produces the P that its
+// first PV needs (o_free).
 #pragma once
 
 #include "attn_tc.cuh"
@@ -238,17 +240,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t bar_q = bar0; // Q buffer 0 landed
     auto bar_kfull = [&](int s) { return bar0 + 8 * (1 + s); };
     auto bar_vfull = [&](int s) { return bar0 + 8 * (1 + kTcStages + s); };
-    auto bar_kempty = [&](int s) { return bar0 + 8 * (1 + 2 * kTcStages + s); };
-    auto bar_vempty = [&](int s) { return bar0 + 8 * (1 + 3 * kTcStages + s); };
-    const uint32_t bar_sfull0 = bar0 + 8 * (1 + 4 * kTcStages); // 2
-    const uint32_t bar_pfull0 = bar_sfull0 + 16;                // 2
-    const uint32_t bar_odone0 = bar_pfull0 + 16;                // 2
+    // A K stage is free again once the QK that read it has completed, which
+    // is what sfull of that tile tracks; a V stage once its PV has completed
+    // (odone of that tile: two barriers for the two V stages).  So the
+    // producers wait on those and the MMA thread commits nothing extra.
+    static_assert(kTcStages == 2, "odone doubles as the V-stage release");
+    const uint32_t bar_sfull0 = bar0 + 8 * (1 + 2 * kTcStages); // kSBufs
+    const uint32_t bar_pfull0 = bar_sfull0 + 8 * kSBufs;        // kSBufs
+    const uint32_t bar_odone0 = bar_pfull0 + 8 * kSBufs;        // 2
     const uint32_t bar_final = bar_odone0 + 16;
-    const uint32_t bar_qfree0 = bar_final + 8; // 2: Q buffer no longer read
-    const uint32_t bar_ofree0 = bar_qfree0 + 16; // 2: O buffer read out
-    const uint32_t bar_qfull1 = bar_ofree0 + 16; // Q buffer 1 landed
-    const uint32_t bar_ifull0 = bar0 + 168;  // 4: work item published
-    const uint32_t bar_iempty0 = bar0 + 200; // 4: work item read by all roles
+    const uint32_t bar_qfree0 = bar_final + 8;  // 2: Q buffer no longer read
+    const uint32_t bar_ofree = bar_qfree0 + 16; // O read out by the epilogue
+    const uint32_t bar_qfull1 = bar_ofree + 8;  // Q buffer 1 landed
+    const uint32_t bar_ifull0 = bar_qfull1 + 8;   // 4: work item published
+    const uint32_t bar_iempty0 = bar_ifull0 + 32; // 4: work item read by all roles
+    static_assert(8 * (1 + 2 * kTcStages) + 16 * kSBufs + 16 + 8 + 16 + 8 + 8 + 64 <= 256,
+                  "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kSmemBar + 256);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kSmemBar + 384);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + kSmemBar + 392);
@@ -260,23 +267,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int s = 0; s < kTcStages; ++s) {
             mbar_init(bar_kfull(s), 1);
             mbar_init(bar_vfull(s), 1);
-            mbar_init(bar_kempty(s), 1);
-            mbar_init(bar_vempty(s), 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kSBufs; ++i) {
             mbar_init(bar_sfull0 + 8 * i, 1);
             mbar_init(bar_pfull0 + 8 * i, 128);
+        }
+        for (int i = 0; i < 2; ++i)
             mbar_init(bar_odone0 + 8 * i, 1);
-        }
         mbar_init(bar_final, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 2; ++i)
             mbar_init(bar_qfree0 + 8 * i, 1);
-            mbar_init(bar_ofree0 + 8 * i, 128);
-        }
+        mbar_init(bar_ofree, 128);
         mbar_init(bar_qfull1, 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_ifull0 + 8 * i, 1);
-            mbar_init(bar_iempty0 + 8 * i, 129); // MMA thread + 128 softmax threads
+            mbar_init(bar_iempty0 + 8 * i, 130); // MMA, V producer, 128 softmax threads
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -291,8 +296,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s0 = tmem;      // S buffers: columns [0, 128), [128, 256)
-    const uint32_t t_o0 = tmem + 256; // O buffers: columns [256, 384), [384, 512)
+    const uint32_t t_s0 = tmem;              // S/P buffers: columns [128 i, 128 i + 128)
+    const uint32_t t_o = tmem + 128 * kSBufs; // O: columns [384, 512)
     auto bar_qfull = [&](int i) { return i ? bar_qfull1 : bar_q; };
 
     Src src;
@@ -342,36 +347,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
 
     if (warp == 4) {
-        // ---------------------------------------------------- TMA producer
+        // ------------------------------------------- TMA producer: Q and K
         if (lane == 0) {
             bool ok = true;
             int si = 0;
             long long g = 0;   // running K/V tile counter
-            long long kiss = 0, viss = 0;
-            // Decode: V of a tile is issued after K of the next one, so the
-            // K load that QK waits for never queues behind a V load (PV
-            // needs V a whole softmax later); measured ~3% faster there.
-            // Forward: V follows its own K at once (deferring it measured
-            // ~1% slower on long sequences).  pv_*: the V load not issued.
-            bool pv = false, pv_skip = false;
-            int pv_ks = 0, pv_head = 0;
-            long long pv_g = 0;
-            auto issue_v = [&]() -> bool {
-                const int s = (int)(pv_g % kTcStages);
-                const uint32_t ph = (uint32_t)((pv_g / kTcStages) & 1) ^ 1u;
-                pv = false;
-                if (pv_skip)
-                    return true;
-                if (pv_g >= kTcStages && !mbar_wait(bar_vempty(s), ph, abort_flag))
-                    return false;
-                mbar_expect_tx(bar_vfull(s), kTileBytes);
-                tma_load_3d(base + kSmemV + s * kTileBytes, &tm_v, 0, pv_ks, pv_head,
-                            bar_vfull(s));
-                tma_load_3d(base + kSmemV + s * kTileBytes + kHalfTileBytes, &tm_v, 64,
-                            pv_ks, pv_head, bar_vfull(s));
-                viss = pv_g + 1;
-                return true;
-            };
+            long long kiss = 0;
             while (ok && next_seg(si, true, ok)) {
                 // Q buffer si & 1 was last read by segment si - 2
                 const int qbuf = si & 1;
@@ -388,33 +369,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const int ks = it < sg.n0 ? sg.lo0 + it * kTcN
                                               : sg.lo1 + (it - sg.n0) * kTcN;
                     const int s = (int)(g % kTcStages);
-                    const uint32_t ph = (uint32_t)((g / kTcStages) & 1) ^ 1u;
-                    if (g >= kTcStages && !(ok = mbar_wait(bar_kempty(s), ph, abort_flag)))
-                        break;
-                    bool skip = false;
-                    if (g == 0 && blockIdx.x == 0 && atomicExch(&g_fault_skip_k, 0) != 0)
-                        skip = true; // injected fault: this tile never arrives
-                    if (!skip) {
-                        mbar_expect_tx(bar_kfull(s), kTileBytes);
-                        tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks,
-                                    sg.kvhead, bar_kfull(s));
-                        tma_load_3d(base + kSmemK + s * kTileBytes + kHalfTileBytes,
-                                    &tm_k, 64, ks, sg.kvhead, bar_kfull(s));
-                        kiss = g + 1;
+                    // stage s was last read by QK_{g-2}
+                    if (g >= kTcStages) {
+                        const long long gp = g - kTcStages;
+                        if (!(ok = mbar_wait(bar_sfull0 + 8 * (int)(gp % kSBufs),
+                                             (uint32_t)((gp / kSBufs) & 1), abort_flag)))
+                            break;
                     }
-                    if (pv && !(ok = issue_v()))
-                        break;
-                    pv = true;
-                    pv_skip = skip;
-                    pv_ks = ks;
-                    pv_head = sg.kvhead;
-                    pv_g = g;
-                    if (KIND == 0 && !(ok = issue_v()))
-                        break;
+                    if (g == 0 && blockIdx.x == 0 && atomicExch(&g_fault_skip_k, 0) != 0)
+                        continue; // injected fault: this tile never arrives
+                    mbar_expect_tx(bar_kfull(s), kTileBytes);
+                    tma_load_3d(base + kSmemK + s * kTileBytes, &tm_k, 0, ks, sg.kvhead,
+                                bar_kfull(s));
+                    tma_load_3d(base + kSmemK + s * kTileBytes + kHalfTileBytes, &tm_k, 64,
+                                ks, sg.kvhead, bar_kfull(s));
+                    kiss = g + 1;
                 }
             }
-            if (ok && pv)
-                ok = issue_v();
             if (KIND == 0) {
                 // this CTA takes no more items; the last CTA resets the pair
                 __threadfence();
@@ -433,8 +404,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 drain(bar_qfull(x & 1), (uint32_t)((x >> 1) & 1));
             for (long long x = kiss > kTcStages ? kiss - kTcStages : 0; x < kiss; ++x)
                 drain(bar_kfull((int)(x % kTcStages)), (uint32_t)((x / kTcStages) & 1));
+        }
+    } else if (warp == 6) {
+        // ---------------------------------------------- TMA producer: V
+        // A warp of its own, so a K load never queues behind a V load that
+        // waits for its stage (and the other way round).
+        if (lane == 0) {
+            bool ok = true;
+            int si = 0;
+            long long g = 0;
+            long long viss = 0;
+            while (ok && next_seg(si, false, ok)) {
+                ++si;
+                for (int it = 0; it < sg.nt; ++it, ++g) {
+                    const int ks = it < sg.n0 ? sg.lo0 + it * kTcN
+                                              : sg.lo1 + (it - sg.n0) * kTcN;
+                    const int s = (int)(g % kTcStages);
+                    // stage s was last read by PV_{g-2}
+                    if (g >= kTcStages &&
+                        !(ok = mbar_wait(bar_odone0 + 8 * (int)(g & 1),
+                                         (uint32_t)(((g - kTcStages) >> 1) & 1), abort_flag)))
+                        break;
+                    mbar_expect_tx(bar_vfull(s), kTileBytes);
+                    tma_load_3d(base + kSmemV + s * kTileBytes, &tm_v, 0, ks, sg.kvhead,
+                                bar_vfull(s));
+                    tma_load_3d(base + kSmemV + s * kTileBytes + kHalfTileBytes, &tm_v, 64,
+                                ks, sg.kvhead, bar_vfull(s));
+                    viss = g + 1;
+                }
+            }
+            const long long c0 = clock64();
             for (long long x = viss > kTcStages ? viss - kTcStages : 0; x < viss; ++x)
-                drain(bar_vfull((int)(x % kTcStages)), (uint32_t)((x / kTcStages) & 1));
+                while (!mbar_try_wait(bar_vfull((int)(x % kTcStages)),
+                                      (uint32_t)((x / kTcStages) & 1)) &&
+                       clock64() - c0 < kWaitCycles) {}
         }
     } else if (warp == 5) {
         // ---------------------------------------------------- MMA issuer
@@ -446,28 +449,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             long long j = 0; // running tile counter
             auto issue_pv = [&](long long jg, bool first) -> bool {
                 const int s = (int)(jg % kTcStages);
-                // O buffer si & 1 was last read out by segment si - 2
-                if (first && si >= 2 &&
-                    !mbar_wait(bar_ofree0 + 8 * (si & 1), (uint32_t)(((si - 2) >> 1) & 1),
-                               abort_flag))
+                const int b = (int)(jg % kSBufs);
+                // O was last read out by the epilogue of segment si - 1
+                if (first && si >= 1 &&
+                    !mbar_wait(bar_ofree, (uint32_t)((si - 1) & 1), abort_flag))
                     return false;
-                if (!mbar_wait(bar_pfull0 + 8 * (jg & 1), (uint32_t)((jg >> 1) & 1), abort_flag))
+                if (!mbar_wait(bar_pfull0 + 8 * b, (uint32_t)((jg / kSBufs) & 1), abort_flag))
                     return false;
                 if (!mbar_wait(bar_vfull(s), (uint32_t)((jg / kTcStages) & 1), abort_flag))
                     return false;
                 tc_fence_after();
                 const uint32_t vb = base + kSmemV + s * kTileBytes;
-                const uint32_t tp = t_s0 + (uint32_t)(jg & 1) * 128;
+                const uint32_t tp = t_s0 + (uint32_t)b * 128;
 #pragma unroll
                 for (int kk = 0; kk < kTcN / 16; ++kk) {
                     uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, kHalfTileBytes, 1024);
-                    tc_mma_ts(t_o0 + (uint32_t)(si & 1) * 128, tp + kk * 8, bdesc, idesc_pv,
-                              (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(t_o, tp + kk * 8, bdesc, idesc_pv, (!first || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(bar_odone0 + 8 * (jg & 1));
-                tc_commit(bar_vempty(s));
                 return true;
             };
+            // Issue order QK_t, PV_{t-kLook} inside a segment; the last PVs
+            // of a segment go out before the next segment's QKs, so its
+            // epilogue is not held up by the next segment's loads.  Forward
+            // (kLook = 2): with kSBufs = 3 S/P buffers the QK two tiles ahead
+            // never waits for the softmax of tile t - 2, so the softmax warps
+            // find the next S ready.  Decode (kLook = 1): HBM-bound, so PV
+            // goes out as early as possible to turn the V ring over faster.
+            // The buffer QK_t overwrites held P_{t-3}, whose PV was issued
+            // before it (tcgen05.mma from one thread execute in issue order).
+            constexpr int kLook = KIND == 0 ? 2 : 1;
+            static_assert(kLook < kSBufs, "QK would overwrite a P not yet consumed");
             while (ok && next_seg(si, false, ok)) {
                 if (!(ok = mbar_wait(bar_qfull(si & 1), (uint32_t)((si >> 1) & 1), abort_flag)))
                     break;
@@ -480,7 +492,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     tc_fence_after();
                     const uint32_t kb = base + kSmemK + s * kTileBytes;
                     const uint32_t qb = base + kSmemQ + (si & 1) * kTileBytes;
-                    const uint32_t ts = t_s0 + (uint32_t)(jg & 1) * 128;
+                    const int b = (int)(jg % kSBufs);
+                    const uint32_t ts = t_s0 + (uint32_t)b * 128;
 #pragma unroll
                     for (int kk = 0; kk < kTcD / 16; ++kk) {
                         const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
@@ -488,15 +501,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                   smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
                                   kk > 0 ? 1u : 0u);
                     }
-                    tc_commit(bar_sfull0 + 8 * (jg & 1));
-                    tc_commit(bar_kempty(s));
+                    tc_commit(bar_sfull0 + 8 * b);
                     if (jj == sg.nt - 1)
                         tc_commit(bar_qfree0 + 8 * (si & 1)); // Q buffer no longer read
-                    if (jj >= 1)
-                        ok = issue_pv(jg - 1, jj == 1);
+                    if (jj >= kLook && !(ok = issue_pv(jg - kLook, jj == kLook)))
+                        break;
                 }
-                if (ok)
-                    ok = issue_pv(j + sg.nt - 1, sg.nt == 1);
+                for (int t = sg.nt > kLook ? sg.nt - kLook : 0; ok && t < sg.nt; ++t)
+                    ok = issue_pv(j + t, t == 0);
                 j += sg.nt;
                 ++si;
             }
@@ -517,7 +529,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!got || !ok)
                 break;
-            const uint32_t t_o = t_o0 + (uint32_t)(si & 1) * 128; // this segment's O
             const int rl = min(row, sg.nrows - 1);
             Span sp;
             if (KIND == 0) {
@@ -536,12 +547,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 const int khi = r0 ? sg.hi0 : sg.hi1;
                 const int flo = r0 ? sg.flo0 : sg.flo1;
                 const int fhi = r0 ? sg.fhi0 : sg.fhi1;
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull0 + 8 * (jg & 1),
-                                                       (uint32_t)((jg >> 1) & 1), abort_flag));
+                const int sb = (int)(jg % kSBufs);
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull0 + 8 * sb,
+                                                       (uint32_t)((jg / kSBufs) & 1), abort_flag));
                 if (!ok)
                     break;
                 tc_fence_after();
-                const uint32_t ts = t_s0 + (uint32_t)(jg & 1) * 128 + lane_off;
+                const uint32_t ts = t_s0 + (uint32_t)sb * 128 + lane_off;
                 uint32_t sr[128];
                 tmem_ld32(ts + 0, sr + 0);
                 tmem_ld32(ts + 32, sr + 32);
@@ -613,7 +625,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar_pfull0 + 8 * (jg & 1));
+                mbar_arrive(bar_pfull0 + 8 * sb);
             }
             if (!ok)
                 break;
@@ -670,7 +682,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (KIND == 1 && !to_out && sg.last_cta >= 0 && row == 0)
                 p.cut_desc[blockIdx.x] = make_int4(sg.nrows, sg.last_cta, sg.out_row0, 0);
             tc_fence_before();
-            mbar_arrive(bar_ofree0 + 8 * (si & 1));
+            mbar_arrive(bar_ofree);
             j += sg.nt;
             ++si;
         }
