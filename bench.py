@@ -54,11 +54,13 @@ def flush_l2(flush, i):
 HOST_COVER_CYCLES = 400000  # ~0.2 ms GPU sleep queued before each timed step
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel, from the ncu captures summarised under profiles/
-# (bd_mma_attn_kernel_fwd_training_shape.md,
-# bd_mma_attn_kernel_decode_denoise.md); None whenever the kernel has changed
-# since those counters were taken.
-FWD_TRAFFIC_BYTES = None
-DECODE_TRAFFIC_BYTES = None
+# (bd_tc_persist_kernel_fwd_training_shape.md: 201,656,064 read + 100,738,816
+# written; bd_tc_persist_kernel_decode.md: 543,351,552 read + 3,873,792
+# written by the denoising-decode attention kernel, whose combine launch
+# moves no tile data in whole-unit mode).  Set back to None whenever the
+# kernel changes after those counters were taken.
+FWD_TRAFFIC_BYTES = 302394880
+DECODE_TRAFFIC_BYTES = 547225344
 
 
 def fwd_flops(s) -> int:
@@ -309,7 +311,7 @@ def run_ours(args):
                              "frac_of_measured_bf16": round(tf / tf_burst, 4)}
             del qd, kd, vd, o, ls
 
-    # ---- block decode workloads (split-KV kernel + LSE combine per call)
+    # ---- block decode workloads (stream-K attention kernel + combine per call)
     dec_roof = None
     if only in ("all", "decode"):
         for sd in (bd_inputs.DEC_DENOISE, bd_inputs.DEC_VERIFY):
@@ -336,7 +338,7 @@ def run_ours(args):
                             "frac": round(gbs / hbm, 4),
                             "traffic": DECODE_TRAFFIC_BYTES,
                             "peak_source": peak_kind,
-                            "kernels": "split-KV + LSE combine"}
+                            "kernels": "stream-K attention + combine"}
             del qd, kcd, vcd, o, ls, ws
     clocks = sampler.stop()
 
