@@ -40,7 +40,7 @@ constexpr int kSBufs = 3;
 #ifndef BD_EXP2_EMU
 #define BD_EXP2_EMU 1
 #endif
-// evaluate a quarter of the FULL-tile exponentials with ex2_poly2
+// evaluate a quarter of each tile's exponentials with ex2_poly2
 constexpr bool kEmuExp2 = BD_EXP2_EMU != 0;
 constexpr int kTileBytes = kTcN * kTcD * 2;          // 32 KB
 constexpr int kHalfTileBytes = kTileBytes / 2;       // one 64-column box
