@@ -67,8 +67,11 @@ constexpr long long kWaitCycles = 4000000000LL;      // ~2 s at 2 GHz
 constexpr int kSmemQ = 0;                      // two Q buffers
 constexpr int kSmemK = kSmemQ + 2 * kTileBytes;
 constexpr int kSmemV = kSmemK + kTcStages * kTileBytes;
-constexpr int kSmemBar = kSmemV + kTcStages * kTileBytes;
+// epilogue staging: per softmax warp, its 32 output rows of 256 bytes
+constexpr int kSmemEpi = kSmemV + kTcStages * kTileBytes;
+constexpr int kSmemBar = kSmemEpi + 4 * 32 * 256;
 constexpr int kTcSmemBytes = kSmemBar + 512 + 1024; // + alignment slack
+static_assert(kTcSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
 // ---------------------------------------------------------------------------
 // PTX wrappers

@@ -648,12 +648,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             else
                 grow = (size_t)sg.out_row0 + row;
             const size_t prow = ((size_t)blockIdx.x * 2 + sg.slot) * kTcM + row;
+            // Forward: output rows go through this warp's staging area so
+            // that each global store writes two whole rows (512 contiguous
+            // bytes) instead of one 16-byte piece of 32 rows.  Chunk c (16
+            // bytes) of row l sits at l * 256 + ((c ^ (l & 7)) << 4):
+            // conflict-free both for a lane writing its own row and for 16
+            // lanes reading one row.  (Decode writes few output tiles per
+            // CTA; it keeps the per-row stores.)
+            constexpr bool kStage = KIND == 0;
+            const uint32_t epi = base + kSmemEpi + (uint32_t)warp * (32 * 256);
 #pragma unroll
             for (int q4 = 0; q4 < kTcD / 32; ++q4) {
                 uint32_t o[32];
                 tmem_ld32(t_o + lane_off + q4 * 32, o);
                 tmem_wait_ld();
-                if (valid && to_out) {
+                if (kStage) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        const uint32_t c = (uint32_t)(q4 * 4 + i / 8);
+                        const uint32_t a = epi + (uint32_t)lane * 256 + ((c ^ (uint32_t)(lane & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv))
+                                     : "memory");
+                    }
+                } else if (valid && to_out) {
                     uint4 *orow = reinterpret_cast<uint4 *>(p.out + grow * kTcD);
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
@@ -672,6 +693,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                             __uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
                             __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
                 }
+            }
+            if (kStage) {
+                __syncwarp();
+                const size_t row0 = grow - (size_t)row + (size_t)warp * 32; // this warp's first row
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 2 * i + (lane >> 4); // row within the warp's 32
+                    const uint32_t cc = (uint32_t)(lane & 15);
+                    uint32_t x0, x1, x2, x3;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                                 : "r"(epi + (uint32_t)r * 256 + ((cc ^ (uint32_t)(r & 7)) << 4))
+                                 : "memory");
+                    if (warp * 32 + r < sg.nrows)
+                        reinterpret_cast<uint4 *>(p.out + (row0 + r) * kTcD)[cc] =
+                            make_uint4(x0, x1, x2, x3);
+                }
+                __syncwarp();
             }
             if (valid) {
                 if (to_out)
