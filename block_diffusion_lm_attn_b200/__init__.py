@@ -106,6 +106,15 @@ def bd_attn_debug_inject_fault(kind):
     return fn(kind)
 
 
+def bd_attn_debug_set_grid(ctas):
+    """Test hook (include/bd_attn_debug.h): cap the grid of the persistent
+    head-dim-128 kernels at `ctas` CTAs (0 restores one CTA per SM)."""
+    fn = load().bd_attn_debug_set_grid
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int]
+    return fn(ctas)
+
+
 # ---------------------------------------------------------------------------
 # torch-tensor conveniences
 

@@ -41,15 +41,20 @@ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Grid cap set by bd_attn_debug_set_grid (0: none).
+std::atomic<int> g_grid_cap{0};
+
 int persistent_grid()
 {
     int dev = 0, sms = kMaxGrid;
+    int g = kMaxGrid;
     if (cudaGetDevice(&dev) == cudaSuccess &&
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) ==
             cudaSuccess &&
         sms > 0)
-        return sms < kMaxGrid ? sms : kMaxGrid;
-    return kMaxGrid;
+        g = sms < kMaxGrid ? sms : kMaxGrid;
+    const int cap = g_grid_cap.load();
+    return cap > 0 && cap < g ? cap : g;
 }
 
 // Decode launch plan.  A pure function of the sizes, so the workspace query
@@ -445,6 +450,14 @@ bd_status bd_attn_debug_inject_fault(int kind)
     return cudaMemcpyToSymbol(bd::g_fault_skip_k, &kind, sizeof kind) == cudaSuccess
                ? BD_OK
                : BD_ERR_CUDA;
+}
+
+bd_status bd_attn_debug_set_grid(int ctas)
+{
+    if (ctas < 0 || ctas > kMaxGrid)
+        return BD_ERR_INVALID_ARG;
+    g_grid_cap.store(ctas);
+    return BD_OK;
 }
 
 bd_status bd_attn_get_device_status(cudaStream_t stream)

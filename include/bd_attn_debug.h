@@ -1,6 +1,7 @@
 /*
- * bd_attn_debug.h -- test hook of libbdattn.so for the failure-detection
- * path (no counterpart on the source pages).
+ * bd_attn_debug.h -- test hooks of libbdattn.so (no counterpart on the
+ * source pages): the failure-detection path, and the grid size of the
+ * persistent kernels.
  *
  * Every wait inside the tensor-core kernels is bounded: when one runs out,
  * the kernel records BD_ERR_DEVICE_TIMEOUT in the device status word (read
@@ -28,6 +29,17 @@ extern "C" {
  * kind, or BD_ERR_CUDA.
  */
 BD_API bd_status bd_attn_debug_inject_fault(int kind);
+
+/*
+ * Caps the grid of the persistent head-dim-128 kernels (bd_attn_fwd and
+ * bd_attn_decode with d = 128) at `ctas` CTAs for every later launch from
+ * any thread, so tests can run the forward's dynamic hand-out and the
+ * decode's stream-K split and combine at grid sizes other than one CTA per
+ * SM.  ctas = 0 restores the default (one CTA per SM, at most 148).
+ * Results are the same at any grid size up to rounding order.  Returns
+ * BD_OK, or BD_ERR_INVALID_ARG for ctas < 0 or ctas > 148.
+ */
+BD_API bd_status bd_attn_debug_set_grid(int ctas);
 
 #ifdef __cplusplus
 }

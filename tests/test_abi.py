@@ -113,3 +113,9 @@ def test_product_path_does_not_touch_the_oracle():
 
 def test_fault_hook_rejects_unknown_kind(lib):
     assert bd.bd_attn_debug_inject_fault(7) == bd.BD_ERR_INVALID_ARG
+
+
+def test_grid_hook_rejects_out_of_range(lib):
+    assert bd.bd_attn_debug_set_grid(-1) == bd.BD_ERR_INVALID_ARG
+    assert bd.bd_attn_debug_set_grid(149) == bd.BD_ERR_INVALID_ARG
+    assert bd.bd_attn_debug_set_grid(0) == bd.BD_OK
