@@ -621,7 +621,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
                 float rsum[4] = {0.f, 0.f, 0.f, 0.f};
-                softmax_p_tile<kEmuExp2>(s, sl2, nm, ts, rsum);
+                // the FMA-pipe exponential relieves the special-function
+                // unit where the softmax paces the tensor pipe (forward); the
+                // HBM-bound decode measured faster without it
+                softmax_p_tile<KIND == 0 && kEmuExp2>(s, sl2, nm, ts, rsum);
                 l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
                 tmem_wait_st();
                 tc_fence_before();
