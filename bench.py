@@ -54,13 +54,13 @@ def flush_l2(flush, i):
 HOST_COVER_CYCLES = 400000  # ~0.2 ms GPU sleep queued before each timed step
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel, from the ncu captures summarised under profiles/
-# (bd_tc_persist_kernel_fwd_training_shape.md: 201,656,064 read + 100,738,816
-# written; bd_tc_persist_kernel_decode.md: 543,351,552 read + 3,873,792
+# (bd_tc_persist_kernel_fwd_training_shape.md: 201,396,480 read + 105,713,920
+# written; bd_tc_persist_kernel_decode.md: 543,351,040 read + 7,544,064
 # written by the denoising-decode attention kernel, whose combine launch
 # moves no tile data in whole-unit mode).  Set back to None whenever the
 # kernel changes after those counters were taken.
-FWD_TRAFFIC_BYTES = 302394880
-DECODE_TRAFFIC_BYTES = 547225344
+FWD_TRAFFIC_BYTES = 307110400
+DECODE_TRAFFIC_BYTES = 550895104
 
 
 def fwd_flops(s) -> int:
