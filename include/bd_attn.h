@@ -77,6 +77,13 @@ typedef enum {
  * size <= 0, Hq % Hkv != 0, L % b != 0, or a non-finite/non-positive scale;
  * BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA if the launch
  * fails.
+ *
+ * Concurrency (d = 128): the launch is one persistent CTA per SM that takes
+ * its work items from one of 64 counter pairs in device memory, chosen
+ * round-robin when the call is made (and so fixed inside a captured CUDA
+ * graph) and reset by the launch's last CTA.  Launches sharing a pair must
+ * not overlap in time: keep fewer than 64 calls in flight per device, and do
+ * not run two replays of one captured graph at the same time.
  */
 BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
                       float *lse, int B, int Hq, int Hkv, int L, int b, int d,
