@@ -30,10 +30,7 @@ constexpr int kTcThreads = 224; // 4 softmax warps, K producer, MMA, V producer
 constexpr int kTcM = 128;     // query rows per CTA
 constexpr int kTcN = 128;     // keys per K/V tile
 constexpr int kTcD = 128;     // head dim
-#ifndef BD_TC_STAGES
-#define BD_TC_STAGES 2
-#endif
-constexpr int kTcStages = BD_TC_STAGES; // K/V ring depth
+constexpr int kTcStages = 2; // depth of the K ring and of the V ring
 // TMEM S/P buffers of the persistent kernel (128 columns each; O takes the
 // remaining 128 of the 512)
 constexpr int kSBufs = 3;
