@@ -1,0 +1,537 @@
+// Persistent tcgen05 block-diffusion attention, training/prefill form, two
+// query tiles per CTA.
+//
+// A work item is one 128-row query tile of two query heads that read the
+// same kv-head (heads 2i and 2i + 1 of a GQA group): their key ranges and
+// masks are identical, so every K/V tile brought into shared memory serves
+// 256 query rows.  Two softmax warpgroups, one per query tile, alternate on
+// the tensor pipe: while one computes P from its S, the tensor cores run the
+// other's PV and next QK, so each MMA wait covers twice the work of the
+// one-tile kernel and K/V traffic from L2 halves.
+//
+// Roles: warps 0-3 softmax and epilogue of tile A (thread t = row t = TMEM
+// lane t), warps 4-7 the same for tile B, warp 8 TMA producer of Q and K
+// (and the work-item fetch), warp 9 MMA issuer, warp 10 TMA producer of V,
+// warp 11 idle.  setmaxnreg moves registers from warpgroup 2 to the two
+// softmax warpgroups.
+//
+// TMEM: S_A columns [0, 128), S_B [128, 256), O_A [256, 384), O_B [384, 512);
+// P (bf16) overwrites its own S.  Shared memory: the two Q tiles of the
+// current item (one buffer), two K and two V stages, per-warp output
+// staging, barriers.
+//
+// MMA issue order per key tile j (the chains of A and B interleave):
+//   PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
+// so QK_A(j+1) overwrites S_A only after PV_A(j) -- which read P_A(j) from
+// it -- was issued (tcgen05.mma from one thread execute in issue order).
+#pragma once
+
+#include "attn_tc_persist.cuh"
+
+namespace bd {
+
+constexpr int kPairThreads = 384;
+constexpr int kPairRegsSoftmax = 208; // setmaxnreg of warpgroups 0 and 1
+constexpr int kPairRegsOther = 88;    // setmaxnreg of warpgroup 2
+static_assert(2 * 128 * kPairRegsSoftmax + 128 * kPairRegsOther <=
+                  kPairThreads * (65536 / kPairThreads / 8 * 8),
+              "register split above the launch's allocation");
+
+// shared-memory layout (offsets from a 1024-byte aligned base)
+constexpr int kPairSmemQ = 0;                           // tiles A, B
+constexpr int kPairSmemK = kPairSmemQ + 2 * kTileBytes; // 2 stages
+constexpr int kPairSmemV = kPairSmemK + 2 * kTileBytes; // 2 stages
+constexpr int kPairSmemEpi = kPairSmemV + 2 * kTileBytes; // 8 warps x 4 KB
+constexpr int kPairSmemBar = kPairSmemEpi + 8 * 32 * 128;
+constexpr int kPairSmemBytes = kPairSmemBar + 512 + 1024;
+static_assert(kPairSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
+
+// Work item w of the pair kernel: (batch, head pair) = w / R, cost rank
+// r = w % R (0 = heaviest), as FwdSource with head pairs for heads.
+struct PairSeg {
+    int qhead;  // global index (batch * Hq + head) of tile A; tile B is +1
+    int qrow0, nrows, kvhead;
+    int lo0, hi0, lo1, hi1;
+    int flo0, fhi0, flo1, fhi1;
+    int n0, nt;
+};
+
+__device__ __forceinline__ long long pair_items(const PParams &p)
+{
+    return (long long)p.B * (p.Hq / 2) * 2 * p.qtiles;
+}
+
+__device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
+{
+    const int R = 2 * p.qtiles;
+    const int bp = w / R; // batch * (Hq / 2) + pair
+    const int r = w % R;
+    const int idx = p.qtiles - 1 - (r >> 1);
+    const int clean = r & 1;
+    const int half = p.Hq / 2;
+    const int bi = bp / half, pi = bp % half;
+    sg.qrow0 = (clean ? p.L : 0) + idx * kTcM;
+    sg.nrows = min(kTcM, p.L - idx * kTcM);
+    sg.qhead = bi * p.Hq + 2 * pi;
+    sg.kvhead = bi * p.Hkv + (2 * pi) / (p.Hq / p.Hkv);
+    const Span first = fwd_span(p.L, p.b, sg.qrow0);
+    const Span last = fwd_span(p.L, p.b, sg.qrow0 + sg.nrows - 1);
+    sg.lo0 = first.a0; sg.hi0 = last.a1;
+    sg.lo1 = first.a2; sg.hi1 = last.a3;
+    sg.flo0 = last.a0; sg.fhi0 = first.a1;
+    sg.flo1 = last.a2; sg.fhi1 = first.a3;
+    sg.n0 = sg.hi0 > sg.lo0 ? (sg.hi0 - sg.lo0 + kTcN - 1) / kTcN : 0;
+    const int n1 = sg.hi1 > sg.lo1 ? (sg.hi1 - sg.lo1 + kTcN - 1) / kTcN : 0;
+    sg.nt = sg.n0 + n1;
+}
+
+__global__ void __launch_bounds__(kPairThreads, 1)
+    bd_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const PParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + (base - raw_addr);
+
+    const uint32_t bar0 = base + kPairSmemBar;
+    const uint32_t bar_qfull = bar0;          // both Q tiles landed
+    const uint32_t bar_qfree = bar0 + 8;      // every QK of the item retired
+    auto bar_kfull = [&](int s) { return bar0 + 16 + 8 * s; };
+    auto bar_vfull = [&](int s) { return bar0 + 32 + 8 * s; };
+    auto bar_kempty = [&](int s) { return bar0 + 48 + 8 * s; };
+    auto bar_vempty = [&](int s) { return bar0 + 64 + 8 * s; };
+    auto bar_sfull = [&](int x) { return bar0 + 80 + 8 * x; };  // S_x ready
+    auto bar_pfull = [&](int x) { return bar0 + 96 + 8 * x; };  // P_x written
+    auto bar_odone = [&](int x, int par) { return bar0 + 112 + 16 * x + 8 * par; };
+    auto bar_ofree = [&](int x) { return bar0 + 144 + 8 * x; }; // O_x read out
+    const uint32_t bar_final = bar0 + 160;
+    const uint32_t bar_ifull0 = bar0 + 168;  // 4: work item published
+    const uint32_t bar_iempty0 = bar0 + 200; // 4: work item read by all roles
+    volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 256);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 384);
+    volatile uint32_t *tmem_slot =
+        reinterpret_cast<volatile uint32_t *>(sbase + kPairSmemBar + 392);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_qfull, 1);
+        mbar_init(bar_qfree, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+            mbar_init(bar_vempty(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar_sfull(x), 1);
+            mbar_init(bar_pfull(x), 128);
+            mbar_init(bar_odone(x, 0), 1);
+            mbar_init(bar_odone(x, 1), 1);
+            mbar_init(bar_ofree(x), 128);
+        }
+        mbar_init(bar_final, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_ifull0 + 8 * i, 1);
+            mbar_init(bar_iempty0 + 8 * i, 258); // MMA, V producer, 256 softmax threads
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 9) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32((const void *)tmem_slot)), "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    PairSeg sg;
+    // Next item of this CTA, identical for every role: the Q/K producer
+    // takes it from the launch's global counter and publishes it in
+    // item_ring[si % 4]; the other roles read it there.
+    auto next_seg = [&](int si, bool producer, bool &ok) -> bool {
+        const int slot = si & 3;
+        int w;
+        if (producer) {
+            if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
+                                             (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
+                return false;
+            const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
+            w = (long long)t < pair_items(p) ? (int)t : -1;
+            item_ring[slot] = w;
+            mbar_arrive(bar_ifull0 + 8 * slot);
+        } else {
+            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+                return false;
+            w = item_ring[slot];
+            mbar_arrive(bar_iempty0 + 8 * slot);
+        }
+        if (w < 0)
+            return false;
+        pair_item(p, w, sg);
+        return true;
+    };
+    auto key_start = [&](int it) {
+        return it < sg.n0 ? sg.lo0 + it * kTcN : sg.lo1 + (it - sg.n0) * kTcN;
+    };
+
+    if (warp >= 8) {
+    // warpgroup 2 gives registers to the softmax warpgroups; every warp of
+    // it executes this one instruction
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsOther));
+    if (warp == 8) {
+        // ---------------------------------------- TMA producer: Q and K
+        if (lane == 0) {
+            bool ok = true;
+            int si = 0;
+            long long g = 0, kiss = 0;
+            while (ok && next_seg(si, true, ok)) {
+                // the Q buffer was last read by the QKs of item si - 1
+                if (si >= 1 && !(ok = mbar_wait(bar_qfree, (uint32_t)((si - 1) & 1), abort_flag)))
+                    break;
+                mbar_expect_tx(bar_qfull, 2 * kTileBytes);
+                for (int x = 0; x < 2; ++x) {
+                    const uint32_t dst = base + kPairSmemQ + (uint32_t)x * kTileBytes;
+                    tma_load_3d(dst, &tm_q, 0, sg.qrow0, sg.qhead + x, bar_qfull);
+                    tma_load_3d(dst + kHalfTileBytes, &tm_q, 64, sg.qrow0, sg.qhead + x,
+                                bar_qfull);
+                }
+                ++si;
+                for (int it = 0; it < sg.nt; ++it, ++g) {
+                    const int s = (int)(g & 1);
+                    // stage s was last read by QK_A and QK_B of tile g - 2
+                    if (g >= 2 && !(ok = mbar_wait(bar_kempty(s),
+                                                   (uint32_t)((g >> 1) & 1) ^ 1u, abort_flag)))
+                        break;
+                    if (g == 0 && blockIdx.x == 0 && atomicExch(&g_fault_skip_k, 0) != 0)
+                        continue; // injected fault: this tile never arrives
+                    const int ks = key_start(it);
+                    mbar_expect_tx(bar_kfull(s), kTileBytes);
+                    tma_load_3d(base + kPairSmemK + s * kTileBytes, &tm_k, 0, ks, sg.kvhead,
+                                bar_kfull(s));
+                    tma_load_3d(base + kPairSmemK + s * kTileBytes + kHalfTileBytes, &tm_k, 64,
+                                ks, sg.kvhead, bar_kfull(s));
+                    kiss = g + 1;
+                }
+            }
+            // this CTA takes no more items; the last CTA resets the pair
+            __threadfence();
+            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
+                g_sched_next[p.sched_slot] = 0;
+                g_sched_done[p.sched_slot] = 0;
+                __threadfence();
+            }
+            // wait (bounded) for every copy this role issued
+            const long long c0 = clock64();
+            auto drain = [&](uint32_t bar, uint32_t par) {
+                while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}
+            };
+            if (si >= 1)
+                drain(bar_qfull, (uint32_t)((si - 1) & 1));
+            for (long long x = kiss > 2 ? kiss - 2 : 0; x < kiss; ++x)
+                drain(bar_kfull((int)(x & 1)), (uint32_t)((x >> 1) & 1));
+        }
+    } else if (warp == 10) {
+        // ---------------------------------------------- TMA producer: V
+        if (lane == 0) {
+            bool ok = true;
+            int si = 0;
+            long long g = 0, viss = 0;
+            while (ok && next_seg(si, false, ok)) {
+                ++si;
+                for (int it = 0; it < sg.nt; ++it, ++g) {
+                    const int s = (int)(g & 1);
+                    // stage s was last read by PV_A and PV_B of tile g - 2
+                    if (g >= 2 && !(ok = mbar_wait(bar_vempty(s),
+                                                   (uint32_t)((g >> 1) & 1) ^ 1u, abort_flag)))
+                        break;
+                    const int ks = key_start(it);
+                    mbar_expect_tx(bar_vfull(s), kTileBytes);
+                    tma_load_3d(base + kPairSmemV + s * kTileBytes, &tm_v, 0, ks, sg.kvhead,
+                                bar_vfull(s));
+                    tma_load_3d(base + kPairSmemV + s * kTileBytes + kHalfTileBytes, &tm_v, 64,
+                                ks, sg.kvhead, bar_vfull(s));
+                    viss = g + 1;
+                }
+            }
+            const long long c0 = clock64();
+            for (long long x = viss > 2 ? viss - 2 : 0; x < viss; ++x)
+                while (!mbar_try_wait(bar_vfull((int)(x & 1)), (uint32_t)((x >> 1) & 1)) &&
+                       clock64() - c0 < kWaitCycles) {}
+        }
+    } else if (warp == 9) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16(kTcM, kTcN, 0);
+            constexpr uint32_t idesc_pv = idesc_bf16(kTcM, kTcD, 1);
+            bool ok = true;
+            int si = 0;
+            long long j = 0; // running key-tile counter
+            auto issue_qk = [&](int x, long long jg) {
+                const uint32_t kb = base + kPairSmemK + (uint32_t)(jg & 1) * kTileBytes;
+                const uint32_t qb = base + kPairSmemQ + (uint32_t)x * kTileBytes;
+                const uint32_t ts = tmem + (uint32_t)x * 128;
+#pragma unroll
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    tc_mma_ss(ts, smem_desc_sw128(qb + off, 16, 1024),
+                              smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar_sfull(x));
+            };
+            auto issue_pv = [&](int x, long long jg, bool first) {
+                const uint32_t vb = base + kPairSmemV + (uint32_t)(jg & 1) * kTileBytes;
+                const uint32_t tp = tmem + (uint32_t)x * 128;
+                const uint32_t to = tmem + 256 + (uint32_t)x * 128;
+#pragma unroll
+                for (int kk = 0; kk < kTcN / 16; ++kk) {
+                    uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, kHalfTileBytes, 1024);
+                    tc_mma_ts(to, tp + kk * 8, bdesc, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_odone(x, (int)(jg & 1)));
+            };
+            auto wait_k = [&](long long jg) {
+                return mbar_wait(bar_kfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1), abort_flag);
+            };
+            while (ok && next_seg(si, false, ok)) {
+                if (!(ok = mbar_wait(bar_qfull, (uint32_t)(si & 1), abort_flag)))
+                    break;
+                if (!(ok = wait_k(j)))
+                    break;
+                tc_fence_after();
+                issue_qk(0, j);
+                issue_qk(1, j);
+                tc_commit(bar_kempty((int)(j & 1)));
+                if (sg.nt == 1)
+                    tc_commit(bar_qfree);
+                for (int jj = 0; jj < sg.nt && ok; ++jj) {
+                    const long long jg = j + jj;
+                    const bool more = jj + 1 < sg.nt;
+                    // PV_A(jg), then QK_A(jg + 1) into S_A
+                    if (jj == 0 && si >= 1 &&
+                        !(ok = mbar_wait(bar_ofree(0), (uint32_t)((si - 1) & 1), abort_flag)))
+                        break;
+                    if (!(ok = mbar_wait(bar_pfull(0), (uint32_t)(jg & 1), abort_flag)))
+                        break;
+                    if (!(ok = mbar_wait(bar_vfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
+                                         abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_pv(0, jg, jj == 0);
+                    if (more) {
+                        if (!(ok = wait_k(jg + 1)))
+                            break;
+                        tc_fence_after();
+                        issue_qk(0, jg + 1);
+                    }
+                    // PV_B(jg), then QK_B(jg + 1) into S_B
+                    if (jj == 0 && si >= 1 &&
+                        !(ok = mbar_wait(bar_ofree(1), (uint32_t)((si - 1) & 1), abort_flag)))
+                        break;
+                    if (!(ok = mbar_wait(bar_pfull(1), (uint32_t)(jg & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_pv(1, jg, jj == 0);
+                    tc_commit(bar_vempty((int)(jg & 1)));
+                    if (more) {
+                        issue_qk(1, jg + 1);
+                        tc_commit(bar_kempty((int)((jg + 1) & 1)));
+                        if (jj + 2 == sg.nt)
+                            tc_commit(bar_qfree);
+                    }
+                }
+                j += sg.nt;
+                ++si;
+            }
+            tc_commit(bar_final);
+            const long long c0 = clock64();
+            while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
+        }
+    }
+    } else {
+        // -------------------------------------------- softmax + epilogue
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairRegsSoftmax));
+        const int x = warp >> 2;          // 0: tile A, 1: tile B
+        const int wq = warp & 3;          // TMEM lane quarter
+        const int row = threadIdx.x & 127;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t t_s = tmem + (uint32_t)x * 128;
+        const uint32_t t_o = tmem + 256 + (uint32_t)x * 128;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        long long j = 0;
+        int si = 0;
+        for (;;) {
+            const bool got = next_seg(si, false, ok);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!got || !ok)
+                break;
+            const int rl = min(row, sg.nrows - 1);
+            const Span sp = fwd_span(p.L, p.b, sg.qrow0 + rl);
+            float m_used = -INFINITY, l = 0.f;
+            for (int jj = 0; jj < sg.nt; ++jj) {
+                const long long jg = j + jj;
+                const bool r0 = jj < sg.n0;
+                const int ks = key_start(jj);
+                const int khi = r0 ? sg.hi0 : sg.hi1;
+                const int flo = r0 ? sg.flo0 : sg.flo1;
+                const int fhi = r0 ? sg.fhi0 : sg.fhi1;
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(bar_sfull(x), (uint32_t)(jg & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const uint32_t ts = t_s + lane_off;
+                uint32_t sr[128];
+                tmem_ld32(ts + 0, sr + 0);
+                tmem_ld32(ts + 32, sr + 32);
+                tmem_ld32(ts + 64, sr + 64);
+                tmem_ld32(ts + 96, sr + 96);
+                tmem_wait_ld();
+                float s[kTcN];
+#pragma unroll
+                for (int c = 0; c < kTcN; ++c)
+                    s[c] = __uint_as_float(sr[c]);
+                const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
+                if (!full) {
+                    const int e = min(khi, ks + kTcN);
+                    const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
+                    const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
+#pragma unroll
+                    for (int w = 0; w < kTcN / 32; ++w) {
+                        const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                                           range_bits(lo1 - 32 * w, hi1 - 32 * w);
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
+                    }
+                }
+                float mc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mc[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+                for (int c = 16; c < kTcN; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
+                const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]),
+                                       fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+                const float mt = mx * sl2;
+                // lazy rescale (threshold 2^8), warp-uniform TMEM correction
+                const bool need = mt > m_used + 8.f;
+                const bool warp_need = __any_sync(0xffffffffu, need);
+                float c = 1.f;
+                if (need) {
+                    c = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
+                    l *= c;
+                    m_used = mt;
+                }
+                if (jj >= 1 && warp_need) {
+                    const long long jp = jg - 1; // PV_x(jp) done => O_x stable
+                    ok = __all_sync(0xffffffffu,
+                                    mbar_wait(bar_odone(x, (int)(jp & 1)),
+                                              (uint32_t)((jp >> 1) & 1), abort_flag));
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                        uint32_t o[32];
+                        tmem_ld32(t_o + lane_off + q4 * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * c);
+                        tmem_st32(t_o + lane_off + q4 * 32, o);
+                    }
+                }
+                const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+                float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+                softmax_p_tile<kEmuExp2>(s, sl2, nm, ts, rsum);
+                l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_pfull(x));
+            }
+            if (!ok)
+                break;
+            {
+                const long long jl = j + sg.nt - 1; // last PV of the item
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(x, (int)(jl & 1)),
+                                                       (uint32_t)((jl >> 1) & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+            }
+            // ------------------------------------------------ epilogue
+            // Rows go out through this warp's 4 KB staging area, one
+            // 64-column half at a time, so that each global store writes four
+            // 128-byte row pieces instead of 16-byte pieces of 32 rows.  Chunk
+            // c (16 bytes) of row l sits at l * 128 + ((c ^ (l & 7)) << 4).
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+            const size_t head_row0 = (size_t)(sg.qhead + x) * 2 * p.L + sg.qrow0;
+            const uint32_t epi = base + kPairSmemEpi + (uint32_t)warp * (32 * 128);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int q4 = 2 * h + q;
+                    uint32_t o[32];
+                    tmem_ld32(t_o + lane_off + q4 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        const uint32_t cch = (uint32_t)(q * 4 + i / 8);
+                        const uint32_t a = epi + (uint32_t)lane * 128 +
+                                           ((cch ^ (uint32_t)(lane & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv))
+                                     : "memory");
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 4 * i + (lane >> 3); // row within the warp's 32
+                    const uint32_t cc = (uint32_t)(lane & 7);
+                    uint32_t x0, x1, x2, x3;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                                 : "r"(epi + (uint32_t)r * 128 + ((cc ^ (uint32_t)(r & 7)) << 4))
+                                 : "memory");
+                    const int trow = wq * 32 + r;
+                    if (trow < sg.nrows)
+                        reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * kTcD)[h * 8 + cc] =
+                            make_uint4(x0, x1, x2, x3);
+                }
+                __syncwarp();
+            }
+            if (row < sg.nrows)
+                p.lse[head_row0 + row] = lse_v;
+            tc_fence_before();
+            mbar_arrive(bar_ofree(x));
+            j += sg.nt;
+            ++si;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+} // namespace bd

@@ -20,6 +20,11 @@
 #include "attn_mma.cuh"
 #include "attn_tc.cuh"
 #include "attn_tc_persist.cuh"
+#include "attn_tc_pair.cuh"
+
+#ifndef BD_FWD_PAIR
+#define BD_FWD_PAIR 1
+#endif
 #include "bd_common.cuh"
 
 namespace {
@@ -385,10 +390,19 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
             return BD_ERR_CUDA;
         static std::atomic<unsigned int> launches{0};
         p.sched_slot = (int)(launches.fetch_add(1u) % bd::kSchedSlots);
-        const long long items = (long long)B * Hq * 2 * p.qtiles;
+        // two query heads of one GQA group per CTA when the group size is even
+        const bool pair = BD_FWD_PAIR && (Hq / Hkv) % 2 == 0;
+        const long long items = (long long)B * (pair ? Hq / 2 : Hq) * 2 * p.qtiles;
         int G = persistent_grid();
         if (items < G)
             G = (int)items;
+        if (pair) {
+            if (set_smem<bd::bd_tc_pair_kernel>(bd::kPairSmemBytes) != BD_OK)
+                return BD_ERR_CUDA;
+            bd::bd_tc_pair_kernel<<<G, bd::kPairThreads, bd::kPairSmemBytes, stream>>>(mq, mk,
+                                                                                     mv, p);
+            return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+        }
         return launch_persist<0>(mq, mk, mv, p, G, stream);
     }
 
