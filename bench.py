@@ -54,12 +54,12 @@ def flush_l2(flush, i):
 HOST_COVER_CYCLES = 400000  # ~0.2 ms GPU sleep queued before each timed step
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
 # kernel, from the ncu captures summarised under profiles/
-# (bd_tc_persist_kernel_fwd_training_shape.md: 201,396,480 read + 105,713,920
+# (bd_tc_pair_kernel_fwd_training_shape.md: 201,509,376 read + 100,790,528
 # written; bd_tc_persist_kernel_decode.md: 543,351,040 read + 7,544,064
 # written by the denoising-decode attention kernel, whose combine launch
 # moves no tile data in whole-unit mode).  Set back to None whenever the
 # kernel changes after those counters were taken.
-FWD_TRAFFIC_BYTES = None  # forward kernel changed since its capture
+FWD_TRAFFIC_BYTES = 302299904
 DECODE_TRAFFIC_BYTES = 550895104
 
 
