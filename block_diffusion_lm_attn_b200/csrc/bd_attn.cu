@@ -46,6 +46,26 @@ inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 
 inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The paired forward kernel moves registers between its warpgroups with
+// setmaxnreg, which can only hand out what the CTA was launched with: use it
+// only if the compiled kernel's per-thread registers cover the split (a
+// warpgroup asking for more than exists would wait for ever).
+bool pair_kernel_usable()
+{
+    static std::atomic<int> usable{-1};
+    int u = usable.load();
+    if (u < 0) {
+        cudaFuncAttributes a;
+        u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel) == cudaSuccess &&
+             (long long)a.numRegs * bd::kPairThreads >=
+                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther)
+                ? 1
+                : 0;
+        usable.store(u);
+    }
+    return u == 1;
+}
+
 // Grid cap set by bd_attn_debug_set_grid (0: none).
 std::atomic<int> g_grid_cap{0};
 
@@ -391,7 +411,7 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
         static std::atomic<unsigned int> launches{0};
         p.sched_slot = (int)(launches.fetch_add(1u) % bd::kSchedSlots);
         // two query heads of one GQA group per CTA when the group size is even
-        const bool pair = BD_FWD_PAIR && (Hq / Hkv) % 2 == 0;
+        const bool pair = BD_FWD_PAIR && (Hq / Hkv) % 2 == 0 && pair_kernel_usable();
         const long long items = (long long)B * (pair ? Hq / 2 : Hq) * 2 * p.qtiles;
         int G = persistent_grid();
         if (items < G)
