@@ -21,10 +21,6 @@
 #include "attn_tc.cuh"
 #include "attn_tc_persist.cuh"
 #include "attn_tc_pair.cuh"
-
-#ifndef BD_FWD_PAIR
-#define BD_FWD_PAIR 1
-#endif
 #include "bd_common.cuh"
 
 namespace {
@@ -411,7 +407,7 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
         static std::atomic<unsigned int> launches{0};
         p.sched_slot = (int)(launches.fetch_add(1u) % bd::kSchedSlots);
         // two query heads of one GQA group per CTA when the group size is even
-        const bool pair = BD_FWD_PAIR && (Hq / Hkv) % 2 == 0 && pair_kernel_usable();
+        const bool pair = (Hq / Hkv) % 2 == 0 && pair_kernel_usable();
         const long long items = (long long)B * (pair ? Hq / 2 : Hq) * 2 * p.qtiles;
         int G = persistent_grid();
         if (items < G)
