@@ -45,6 +45,8 @@ _i64p = ctypes.POINTER(ctypes.c_int64)
 _i32p = ctypes.POINTER(ctypes.c_int32)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
 _f64p = ctypes.POINTER(ctypes.c_double)
+_f32p = ctypes.POINTER(ctypes.c_float)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 
 
 def _bind(lib):
@@ -63,6 +65,11 @@ def _bind(lib):
     lib.bdo_fwd_row_probs.restype = ctypes.c_int
     lib.bdo_fwd_row_probs.argtypes = [_u16p, _u16p] + [ctypes.c_int] * 6 + [
         ctypes.c_double, ctypes.c_int64, _f64p]
+    lib.bdo_fwd_mask.restype = ctypes.c_int
+    lib.bdo_fwd_mask.argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
+    lib.bdo_sprint_select.restype = ctypes.c_int
+    lib.bdo_sprint_select.argtypes = [_u16p, _i32p, _f32p, _u8p] + [
+        ctypes.c_int] * 4 + [ctypes.c_double] * 3 + [_f64p, _i32p, _i32p]
     lib.bdo_combine.restype = None
     lib.bdo_combine.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _f64p,
                                 _f64p, _f64p]
@@ -142,7 +149,8 @@ def fwd(q, k, v, L: int, b: int, scale: float, rows=None, lib=None):
 def decode(q_blk, k_cache, v_cache, cache_len, mode: int, scale: float,
            rows=None, lib=None):
     """Block-decode form.  q_blk: [B,Hq,b,d]; caches [B,Hkv,S_cap,d];
-    cache_len: int sequence of B.  Returns fp64 (out, lse) shaped
+    cache_len: int sequence of B; mode 0 (bidirectional block), 1 (causal
+    block) or 2 (prefix only).  Returns fp64 (out, lse) shaped
     [B,Hq,b,d], [B,Hq,b] (or [n,d], [n] for ``rows``)."""
     lib = lib or load()
     B, Hq, b, d = q_blk.shape
@@ -198,3 +206,41 @@ def combine(o_parts, lse_parts, lib=None):
     lib.bdo_combine(n, d, _ptr(o, _f64p), _ptr(l_, _f64p), _ptr(out, _f64p),
                     _ptr(lse, _f64p))
     return out, float(lse[0])
+
+
+def fwd_mask(L: int, b: int, lib=None) -> np.ndarray:
+    """The training/prefill visibility predicate as a dense [2L, 2L] bool
+    matrix (row = query position, column = key position)."""
+    lib = lib or load()
+    m = np.empty((2 * L, 2 * L), np.uint8)
+    if lib.bdo_fwd_mask(L, b, _ptr(m, _u8p)) != 0:
+        raise ValueError("oracle mask rejected its arguments")
+    return m.astype(bool)
+
+
+def sprint_select(k_cache, cache_len, conf, modality, alpha=0.5,
+                  keep_text=1.0, keep_image=0.8, lib=None):
+    """Sparse prefix retention scores and kept positions.
+
+    k_cache [B,Hkv,S_cap,d] bf16; cache_len [B]; conf [B,S_cap] fp32 top-1
+    confidences; modality [B,S_cap] uint8 (0 text, else image).  Returns
+    (score [B,S_cap] fp64, kept [B,S_cap] int32 -- kept positions in order,
+    then -1 --, new_len [B] int32)."""
+    lib = lib or load()
+    B, Hkv, S_cap, d = k_cache.shape
+    kb = _bits(k_cache)
+    lens = np.ascontiguousarray(np.asarray(cache_len, dtype=np.int32))
+    cf = np.ascontiguousarray(np.asarray(conf, dtype=np.float32))
+    md = np.ascontiguousarray(np.asarray(modality, dtype=np.uint8))
+    assert lens.shape == (B,) and cf.shape == (B, S_cap) and md.shape == (B, S_cap)
+    score = np.empty((B, S_cap), np.float64)
+    kept = np.empty((B, S_cap), np.int32)
+    new_len = np.empty((B,), np.int32)
+    rc = lib.bdo_sprint_select(_ptr(kb, _u16p), _ptr(lens, _i32p),
+                               _ptr(cf, _f32p), _ptr(md, _u8p), B, Hkv, d,
+                               S_cap, float(alpha), float(keep_text),
+                               float(keep_image), _ptr(score, _f64p),
+                               _ptr(kept, _i32p), _ptr(new_len, _i32p))
+    if rc != 0:
+        raise ValueError("oracle sprint_select rejected its arguments")
+    return score, kept, new_len

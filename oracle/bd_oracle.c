@@ -30,6 +30,19 @@
  *    "draft bidirectionally, verify causally over the same KV cache" flow of
  *    the same article, section 2 "Linear Speculative Decoding", and of
  *    "Nemotron-Labs-Diffusion-VLM-8B", section "Multi-mode decoding".
+ *    Mode 2 is cross-attention only: the block rows are the canvas of an
+ *    encoder-decoder model and see the encoder's cache positions
+ *    0..cache_len-1 and nothing of the canvas ("DiffusionGemma" pipeline
+ *    page, introduction and pipeline class description); with cache_len = 0
+ *    such a row has no visible key.
+ *
+ *  - Sparse prefix retention (SPRINT, "LLaDA2.0-Uni", section "SPRINT:
+ *    training-free inference acceleration", paragraph "Sparse Prefix
+ *    Retention"): at the start of a block the cached prefix is pruned once.
+ *    Position i gets the score s_i = alpha * I_i + (1 - alpha) * c_i, where
+ *    I_i = |k_i|_2 / mean_j |k_j|_2 is its mean-normalised key norm and c_i
+ *    the caller's top-1 confidence; each modality keeps its best-scoring
+ *    fraction (images r_img = 0.8, text r_text = 1.0 on the page).
  *
  *  - For each query row: gather its visible key list, s_c = scale * q.k_c,
  *    m = max s, Z = sum exp(s_c - m), out = sum exp(s_c - m) / Z * v_c,
@@ -87,17 +100,39 @@ int bdo_fwd_sees(int L, int b, int r, int c)
 }
 
 /* Visibility predicate of the block-decode form: does block row j (0 <= j < b)
- * see cache position c, given cache_len clean positions before the block? */
+ * see cache position c, given cache_len clean positions before the block?
+ * mode 0: the block sees itself bidirectionally (denoising a draft);
+ * mode 1: causally (verifying it); mode 2: not at all -- the rows are a
+ * decoder canvas that cross-attends to an encoder's cache only ("Diffusion-
+ * Gemma" pipeline page: a bidirectional decoder cross-attends to the KV
+ * cache the causal encoder wrote, to denoise a canvas of canvas_length
+ * tokens). */
 int bdo_decode_sees(int cache_len, int b, int mode, int j, int c)
 {
     if (c < 0)
         return 0;
     if (c < cache_len)
         return 1; /* the whole clean prefix */
+    if (mode == 2)
+        return 0; /* cross-attention only: nothing of the canvas itself */
     if (c < cache_len + b) {
         int jc = c - cache_len; /* row of the block that key c belongs to */
         return mode == 0 ? 1 : (jc <= j);
     }
+    return 0;
+}
+
+/* The training/prefill mask as a dense [2L][2L] 0/1 matrix, cell (r, c) =
+ * bdo_fwd_sees(L, b, r, c).  Returns 0, or -1 on a bad argument. */
+int bdo_fwd_mask(int L, int b, uint8_t *mask)
+{
+    if (L <= 0 || b <= 0 || L % b != 0)
+        return -1;
+    const int N = 2 * L;
+    int r, c;
+    for (r = 0; r < N; ++r)
+        for (c = 0; c < N; ++c)
+            mask[(int64_t)r * N + c] = (uint8_t)bdo_fwd_sees(L, b, r, c);
     return 0;
 }
 
@@ -200,10 +235,10 @@ int bdo_fwd_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 /* Block-decode form.
  * q_blk: [B, Hq, b, d]; k_cache, v_cache: [B, Hkv, S_cap, d] (bf16 bits);
  * cache_len: [B]; the block's own keys sit at cache_len[i]..cache_len[i]+b-1.
- * mode: 0 bidirectional inside the block, 1 causal.
+ * mode: 0 bidirectional inside the block, 1 causal, 2 prefix only.
  * rows: flat ids ((batch * Hq + h) * b + j) or NULL for all; out: [nrows, d],
  * lse: [nrows].  Returns 0, or -1 on a bad argument (including
- * cache_len[i] + b > S_cap). */
+ * cache_len[i] + b > S_cap in modes 0 and 1, cache_len[i] > S_cap in mode 2). */
 int bdo_decode_rows(const uint16_t *q_blk, const uint16_t *k_cache,
                     const uint16_t *v_cache, const int32_t *cache_len, int B,
                     int Hq, int Hkv, int b, int d, int S_cap, int mode,
@@ -212,11 +247,14 @@ int bdo_decode_rows(const uint16_t *q_blk, const uint16_t *k_cache,
 {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
         return -1;
-    if (Hq % Hkv != 0 || (mode != 0 && mode != 1))
+    if (Hq % Hkv != 0 || mode < 0 || mode > 2)
         return -1;
     int i;
+    /* modes 0 and 1 read the block's own keys after the prefix; mode 2 reads
+     * the prefix only */
+    const int own = (mode == 2) ? 0 : b;
     for (i = 0; i < B; ++i)
-        if (cache_len[i] < 0 || (int64_t)cache_len[i] + b > S_cap)
+        if (cache_len[i] < 0 || (int64_t)cache_len[i] + own > S_cap)
             return -1;
     const int64_t total = (int64_t)B * Hq * b;
     if (rows == NULL)
@@ -332,4 +370,120 @@ void bdo_combine(int nparts, int d, const double *o_s, const double *lse_s,
         for (t = 0; t < d; ++t)
             out[t] += w * o_s[(int64_t)s * d + t];
     }
+}
+
+/* ------------------------------------------------------------------------
+ * Sparse prefix retention (SPRINT).
+ *
+ * Readings where the page is silent (stated once here, used below):
+ *  - k_i is the key of position i in this cache across all its kv-heads,
+ *    so |k_i|_2 = sqrt(sum over heads h and dims t of k[h][i][t]^2);
+ *  - the mean in I_i runs over the prefix positions 0..cache_len-1 (the L of
+ *    the page's formula); if it is 0 (an all-zero prefix) every I_i is 0;
+ *  - modality 0 is text, any other value image; a modality with n prefix
+ *    positions keeps floor(r * n + 1/2) of them (r widened to double),
+ *    clamped to [0, n]: the best scores, ties broken by the lower position;
+ *  - the kept positions stay in their original order (stable compaction)
+ *    and become the new prefix.
+ */
+
+typedef struct {
+    double s;
+    int p;
+} bdo_scored;
+
+/* higher score first; equal scores: lower position first */
+static int bdo_scored_cmp(const void *a, const void *b)
+{
+    const bdo_scored *x = (const bdo_scored *)a, *y = (const bdo_scored *)b;
+    if (x->s > y->s)
+        return -1;
+    if (x->s < y->s)
+        return 1;
+    return (x->p > y->p) - (x->p < y->p);
+}
+
+/* Scores and kept positions of the prefix of every sequence.
+ * k_cache: [B, Hkv, S_cap, d] bf16 bits; cache_len: [B];
+ * conf: [B, S_cap] fp32 top-1 confidences; modality: [B, S_cap] (0 text,
+ * else image).  Writes score: [B, S_cap] fp64 (0 beyond the prefix),
+ * kept: [B, S_cap] int32, the kept positions in increasing order followed by
+ * -1, and new_len: [B], their number.  Returns 0, or -1 on a bad argument. */
+int bdo_sprint_select(const uint16_t *k_cache, const int32_t *cache_len,
+                      const float *conf, const uint8_t *modality, int B,
+                      int Hkv, int d, int S_cap, double alpha,
+                      double keep_text, double keep_image, double *score,
+                      int32_t *kept, int32_t *new_len)
+{
+    if (B <= 0 || Hkv <= 0 || d <= 0 || S_cap <= 0)
+        return -1;
+    if (!(alpha >= 0.0 && alpha <= 1.0) || !(keep_text >= 0.0 && keep_text <= 1.0) ||
+        !(keep_image >= 0.0 && keep_image <= 1.0))
+        return -1;
+    int i;
+    for (i = 0; i < B; ++i)
+        if (cache_len[i] < 0 || cache_len[i] > S_cap)
+            return -1;
+    for (i = 0; i < B; ++i) {
+        const int n = cache_len[i];
+        double *sc = score + (int64_t)i * S_cap;
+        int32_t *kp = kept + (int64_t)i * S_cap;
+        int p, h, t, m;
+        /* key norms, then their mean over the prefix */
+        double mean = 0.0;
+        for (p = 0; p < S_cap; ++p)
+            sc[p] = 0.0;
+        for (p = 0; p < n; ++p) {
+            double ss = 0.0;
+            for (h = 0; h < Hkv; ++h) {
+                const uint16_t *row = k_cache + (((int64_t)i * Hkv + h) * S_cap + p) * d;
+                for (t = 0; t < d; ++t) {
+                    double x = bf16_bits_to_double(row[t]);
+                    ss += x * x;
+                }
+            }
+            sc[p] = sqrt(ss); /* |k_p|_2 for now */
+            mean += sc[p];
+        }
+        if (n > 0)
+            mean /= n;
+        /* composite score */
+        for (p = 0; p < n; ++p) {
+            double inorm = mean > 0.0 ? sc[p] / mean : 0.0;
+            sc[p] = alpha * inorm + (1.0 - alpha) * (double)conf[(int64_t)i * S_cap + p];
+        }
+        /* per modality: keep the best floor(r n + 1/2) */
+        char *keep = (char *)calloc((size_t)(n > 0 ? n : 1), 1);
+        bdo_scored *lst = (bdo_scored *)malloc(sizeof(bdo_scored) * (size_t)(n > 0 ? n : 1));
+        for (m = 0; m < 2; ++m) {
+            int cnt = 0;
+            for (p = 0; p < n; ++p) {
+                int is_img = modality[(int64_t)i * S_cap + p] != 0;
+                if (is_img == m) {
+                    lst[cnt].s = sc[p];
+                    lst[cnt].p = p;
+                    ++cnt;
+                }
+            }
+            double r = (m == 0) ? keep_text : keep_image;
+            int64_t want = (int64_t)floor(r * (double)cnt + 0.5);
+            if (want < 0)
+                want = 0;
+            if (want > cnt)
+                want = cnt;
+            qsort(lst, (size_t)cnt, sizeof(bdo_scored), bdo_scored_cmp);
+            for (p = 0; p < want; ++p)
+                keep[lst[p].p] = 1;
+        }
+        int nk = 0;
+        for (p = 0; p < n; ++p)
+            if (keep[p])
+                kp[nk++] = p;
+        for (p = nk; p < S_cap; ++p)
+            kp[p] = -1;
+        new_len[i] = nk;
+        free(keep);
+        free(lst);
+    }
+    return 0;
 }
