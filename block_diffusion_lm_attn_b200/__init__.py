@@ -29,7 +29,9 @@ BD_ERR_CUDA = 3
 BD_ERR_DEVICE_TIMEOUT = 4
 
 EXPORTED = ("bd_attn_fwd", "bd_attn_decode", "bd_attn_decode_workspace_bytes",
-            "bd_attn_get_device_status", "bd_attn_status_string")
+            "bd_attn_get_device_status", "bd_attn_status_string",
+            "bd_spec_accept", "bd_cache_append", "bd_cache_crop",
+            "bd_sprint_prune", "bd_sprint_workspace_bytes")
 
 
 class BdAttnError(RuntimeError):
@@ -64,6 +66,18 @@ def load(path: str = LIB_PATH):
     lib.bd_attn_get_device_status.argtypes = [vp]
     lib.bd_attn_status_string.restype = ctypes.c_char_p
     lib.bd_attn_status_string.argtypes = [i]
+    lib.bd_spec_accept.restype = i
+    lib.bd_spec_accept.argtypes = [vp, vp, vp, i, i, vp]
+    lib.bd_cache_append.restype = i
+    lib.bd_cache_append.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.bd_cache_crop.restype = i
+    lib.bd_cache_crop.argtypes = [vp, i, i, vp]
+    lib.bd_sprint_prune.restype = i
+    lib.bd_sprint_prune.argtypes = [vp, vp, vp, vp, vp, f, f, f, vp, vp, vp,
+                                    vp, vp, i, i, i, i, vp, vp,
+                                    ctypes.c_size_t]
+    lib.bd_sprint_workspace_bytes.restype = ctypes.c_size_t
+    lib.bd_sprint_workspace_bytes.argtypes = [i, i]
     _lib = lib
     return lib
 
@@ -95,6 +109,33 @@ def bd_attn_get_device_status(stream):
 
 def bd_attn_status_string(status):
     return load().bd_attn_status_string(status).decode()
+
+
+def bd_spec_accept(draft, target, n_accept, B, b, stream):
+    return load().bd_spec_accept(draft, target, n_accept, B, b, stream)
+
+
+def bd_cache_append(k_cache, v_cache, cache_len, k_new, v_new, n_new, B, Hkv,
+                    b, d, S_cap, stream):
+    return load().bd_cache_append(k_cache, v_cache, cache_len, k_new, v_new,
+                                  n_new, B, Hkv, b, d, S_cap, stream)
+
+
+def bd_cache_crop(cache_len, B, max_len, stream):
+    return load().bd_cache_crop(cache_len, B, max_len, stream)
+
+
+def bd_sprint_prune(k_cache, v_cache, cache_len, conf, modality, alpha,
+                    keep_text, keep_image, k_out, v_out, kept, new_len, score,
+                    B, Hkv, d, S_cap, stream, workspace, workspace_bytes):
+    return load().bd_sprint_prune(k_cache, v_cache, cache_len, conf, modality,
+                                  alpha, keep_text, keep_image, k_out, v_out,
+                                  kept, new_len, score, B, Hkv, d, S_cap,
+                                  stream, workspace, workspace_bytes)
+
+
+def bd_sprint_workspace_bytes(B, S_cap):
+    return int(load().bd_sprint_workspace_bytes(B, S_cap))
 
 
 def bd_attn_debug_inject_fault(kind):
@@ -157,7 +198,8 @@ def decode(q_blk, k_cache, v_cache, cache_len, mode: int, out=None, lse=None,
     """Block-decode attention on CUDA tensors.
 
     q_blk [B,Hq,b,d]; k_cache, v_cache [B,Hkv,S_cap,d] bf16; cache_len int32
-    [B] on the device; mode 0 bidirectional, 1 causal.  ``workspace`` is an
+    [B] on the device; mode 0 bidirectional, 1 causal, 2 cross-attention to
+    the prefix only.  ``workspace`` is an
     optional uint8 CUDA tensor of at least ``workspace_bytes(...)`` bytes
     (None: the library's own per-device buffer).  Returns (out, lse)."""
     import torch
@@ -185,6 +227,100 @@ def decode(q_blk, k_cache, v_cache, cache_len, mode: int, out=None, lse=None,
     if st != BD_OK:
         raise BdAttnError(st, "bd_attn_decode")
     return out, lse
+
+
+def _check(t, dtype, what):
+    import torch
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError("%s must be a contiguous %s CUDA tensor" % (what, dtype))
+
+
+def spec_accept(draft, target, n_accept=None, stream=None):
+    """Longest matching prefix of draft and target ([B, b] int32 CUDA).
+    Returns n_accept [B] int32 on the device."""
+    import torch
+    _check(draft, torch.int32, "draft")
+    _check(target, torch.int32, "target")
+    B, b = draft.shape
+    if tuple(target.shape) != (B, b):
+        raise ValueError("shape mismatch")
+    if n_accept is None:
+        n_accept = torch.empty(B, dtype=torch.int32, device=draft.device)
+    st = bd_spec_accept(draft.data_ptr(), target.data_ptr(),
+                        n_accept.data_ptr(), B, b, _stream_handle(stream))
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_spec_accept")
+    return n_accept
+
+
+def cache_append(k_cache, v_cache, cache_len, n_new, k_new=None, v_new=None,
+                 stream=None):
+    """Append rows 0..n_new[i]-1 of k_new/v_new [B,Hkv,b,d] (or of the rows
+    already at the cache tail, if None) and advance cache_len, in place."""
+    import torch
+    B, Hkv, S_cap, d = k_cache.shape
+    for t, w in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, torch.bfloat16, w)
+    _check(cache_len, torch.int32, "cache_len")
+    _check(n_new, torch.int32, "n_new")
+    if k_new is None:
+        b = S_cap
+        kp = vp = None
+    else:
+        b = k_new.shape[2]
+        kp, vp = k_new.data_ptr(), v_new.data_ptr()
+    st = bd_cache_append(k_cache.data_ptr(), v_cache.data_ptr(),
+                         cache_len.data_ptr(), kp, vp, n_new.data_ptr(), B,
+                         Hkv, b, d, S_cap, _stream_handle(stream))
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_cache_append")
+
+
+def cache_crop(cache_len, max_len: int, stream=None):
+    import torch
+    _check(cache_len, torch.int32, "cache_len")
+    st = bd_cache_crop(cache_len.data_ptr(), cache_len.numel(), int(max_len),
+                       _stream_handle(stream))
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_cache_crop")
+
+
+def sprint_prune(k_cache, v_cache, cache_len, conf, modality, alpha=0.5,
+                 keep_text=1.0, keep_image=0.8, k_out=None, v_out=None,
+                 want_score=False, workspace=None, stream=None):
+    """Sparse prefix retention on CUDA tensors.  Returns (k_out, v_out,
+    kept [B,S_cap] int32, new_len [B] int32, score [B,S_cap] fp64 or None)."""
+    import torch
+    B, Hkv, S_cap, d = k_cache.shape
+    for t, w in ((k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, torch.bfloat16, w)
+    _check(cache_len, torch.int32, "cache_len")
+    _check(conf, torch.float32, "conf")
+    _check(modality, torch.uint8, "modality")
+    dev = k_cache.device
+    if k_out is None:
+        k_out = torch.empty_like(k_cache)
+    if v_out is None:
+        v_out = torch.empty_like(v_cache)
+    kept = torch.empty((B, S_cap), dtype=torch.int32, device=dev)
+    new_len = torch.empty(B, dtype=torch.int32, device=dev)
+    score = (torch.zeros((B, S_cap), dtype=torch.float64, device=dev)
+             if want_score else None)
+    nb = bd_sprint_workspace_bytes(B, S_cap)
+    if workspace is None:
+        workspace = torch.empty(nb, dtype=torch.uint8, device=dev)
+    st = bd_sprint_prune(k_cache.data_ptr(), v_cache.data_ptr(),
+                         cache_len.data_ptr(), conf.data_ptr(),
+                         modality.data_ptr(), float(alpha), float(keep_text),
+                         float(keep_image), k_out.data_ptr(), v_out.data_ptr(),
+                         kept.data_ptr(), new_len.data_ptr(),
+                         score.data_ptr() if score is not None else None,
+                         B, Hkv, d, S_cap, _stream_handle(stream),
+                         workspace.data_ptr(),
+                         workspace.numel() * workspace.element_size())
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_sprint_prune")
+    return k_out, v_out, kept, new_len, score
 
 
 def workspace_bytes(B, Hq, Hkv, b, d, S_cap) -> int:

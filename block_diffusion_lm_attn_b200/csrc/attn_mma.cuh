@@ -109,7 +109,7 @@ __device__ __forceinline__ Span decode_span(const MmaParams &p, const Plan &pl,
                                             int rloc)
 {
     int j = (pl.row0 + rloc) % p.b;
-    int hi = pl.len + (p.mode == 0 ? p.b : j + 1);
+    int hi = pl.len + (p.mode == 0 ? p.b : p.mode == 1 ? j + 1 : 0);
     int s0 = pl.split * p.chunk;
     Span s;
     s.a0 = s0; s.a1 = min(hi, s0 + p.chunk); s.a2 = 0; s.a3 = 0;
@@ -142,9 +142,10 @@ __device__ __forceinline__ bool make_plan(const MmaParams &p, Plan &pl)
         const int group = p.Hq / p.Hkv;
         const int len = p.cache_len[bi];
         const int s = blockIdx.x;
-        if (len < 0 || (long long)len + p.b > p.nkeys)
+        const int own = p.mode == 2 ? 0 : p.b; // keys past the prefix
+        if (len < 0 || (long long)len + own > p.nkeys)
             return false; // reported by the combine kernel
-        const int total = len + p.b;
+        const int total = len + own;
         if (s * p.chunk >= total)
             return false;
         pl.len = len;
@@ -400,7 +401,8 @@ __global__ void __launch_bounds__(256)
     const int len = p.cache_len[bi];
     constexpr int PER = D / 32;
     bf16 *orow = p.out + (size_t)row * D;
-    if (len < 0 || (long long)len + p.b > p.nkeys) {
+    const int own = p.mode == 2 ? 0 : p.b; // keys past the prefix
+    if (len < 0 || (long long)len + own > p.nkeys) {
         for (int t = 0; t < PER; ++t)
             orow[lane * PER + t] = __float2bfloat16_rn(NAN);
         if (lane == 0) {
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(256)
         }
         return;
     }
-    const int ns = (len + p.b + p.chunk - 1) / p.chunk;
+    const int ns = (len + own + p.chunk - 1) / p.chunk;
     float mx = -INFINITY;
     for (int s = 0; s < ns; ++s)
         mx = fmaxf(mx, p.part_lse[(size_t)s * rows_all + row]);

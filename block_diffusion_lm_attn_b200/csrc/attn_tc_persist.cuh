@@ -62,12 +62,21 @@ struct Seg {
                         // units that start in this CTA's range), else -1
 };
 
-// Number of 128-key tiles of one decode unit (0 for an invalid length).
-__device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap)
+// Keys a decode row may see past the prefix: the block itself in modes 0
+// and 1, nothing in mode 2 (cross-attention to the prefix only).
+__device__ __forceinline__ int decode_own_keys(int b, int mode)
 {
-    if (len < 0 || (long long)len + b > S_cap)
-        return 0;
-    return (len + b + kTcN - 1) / kTcN;
+    return mode == 2 ? 0 : b;
+}
+
+// Number of 128-key tiles of one decode unit: -1 for an invalid length,
+// 0 for an empty prefix in mode 2.
+__device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap, int mode)
+{
+    const int own = decode_own_keys(b, mode);
+    if (len < 0 || (long long)len + own > S_cap)
+        return -1;
+    return (len + own + kTcN - 1) / kTcN;
 }
 
 // ----------------------------------------------------------------------------
@@ -147,7 +156,7 @@ struct DecSource {
     __device__ void load_seq(const PParams &p)
     {
         len = seq < p.B ? p.cache_len[seq] : 0;
-        seq_tiles = seq < p.B ? decode_unit_tiles(len, p.b, p.nkeys) : 0;
+        seq_tiles = seq < p.B ? max(0, decode_unit_tiles(len, p.b, p.nkeys, p.mode)) : 0;
     }
     __device__ void init(const PParams &p)
     {
@@ -155,7 +164,7 @@ struct DecSource {
         T = 0;
         int maxt = 0;
         for (int i = 0; i < p.B; ++i) {
-            const int ti = decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
+            const int ti = max(0, decode_unit_tiles(p.cache_len[i], p.b, p.nkeys, p.mode));
             T += (long long)ups * ti;
             maxt = max(maxt, ti);
         }
@@ -168,8 +177,8 @@ struct DecSource {
             const int us = u / ups;
             long long base = 0;
             for (int i = 0; i < p.B && i < us; ++i)
-                base += (long long)ups * decode_unit_tiles(p.cache_len[i], p.b, p.nkeys);
-            const int ti = us < p.B ? decode_unit_tiles(p.cache_len[us], p.b, p.nkeys) : 0;
+                base += (long long)ups * max(0, decode_unit_tiles(p.cache_len[i], p.b, p.nkeys, p.mode));
+            const int ti = us < p.B ? max(0, decode_unit_tiles(p.cache_len[us], p.b, p.nkeys, p.mode)) : 0;
             t0 = t = base + (long long)(u % ups) * ti;
             t1 = t + ti;
         } else {
@@ -200,7 +209,7 @@ struct DecSource {
         sg.qrow0 = rt * kTcM;
         sg.nrows = min(kTcM, p.rows_unit - rt * kTcM);
         sg.lo0 = kt0 * kTcN;
-        sg.hi0 = min((kt0 + n) * kTcN, len + p.b);
+        sg.hi0 = min((kt0 + n) * kTcN, len + decode_own_keys(p.b, p.mode));
         sg.lo1 = sg.hi1 = 0;
         sg.flo0 = 0;
         sg.fhi0 = len + (p.mode == 0 ? p.b : 0);
@@ -536,7 +545,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             } else {
                 const int jr = (sg.qrow0 + rl) % p.b;
                 sp.a0 = 0;
-                sp.a1 = sg.len + (p.mode == 0 ? p.b : jr + 1);
+                sp.a1 = sg.len + (p.mode == 0 ? p.b : p.mode == 1 ? jr + 1 : 0);
                 sp.a2 = sp.a3 = 0;
             }
             float m_used = -INFINITY, l = 0.f;
@@ -760,18 +769,23 @@ __global__ void __launch_bounds__(256)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int R = kCombineRowsPerWarp;
 
-    if (rg == 0) { // invalid sequences (i % G == c): NaN rows; the
-                   // attention kernel writes nothing for them
+    if (rg == 0) { // sequences with no key tile (i % G == c), for which the
+                   // attention kernel writes nothing: an invalid length gives
+                   // NaN rows, an empty prefix in mode 2 rows with no visible
+                   // key (out 0, lse -inf)
         for (int i = c; i < p.B; i += gridDim.x) {
-            if (decode_unit_tiles(p.cache_len[i], p.b, p.nkeys) != 0)
+            const int tiles = decode_unit_tiles(p.cache_len[i], p.b, p.nkeys, p.mode);
+            if (tiles > 0)
                 continue;
+            const float fill = tiles < 0 ? NAN : 0.f;
+            const float lfill = tiles < 0 ? NAN : -INFINITY;
             for (int r = threadIdx.x; r < p.Hq * p.b; r += blockDim.x) {
                 const size_t orow = (size_t)i * p.Hq * p.b + r;
                 for (int t = 0; t < kTcD; ++t)
-                    p.out[orow * kTcD + t] = __float2bfloat16_rn(NAN);
-                p.lse[orow] = NAN;
+                    p.out[orow * kTcD + t] = __float2bfloat16_rn(fill);
+                p.lse[orow] = lfill;
             }
-            if (threadIdx.x == 0)
+            if (threadIdx.x == 0 && tiles < 0)
                 raise_device_code(DEV_BAD_CACHE_LEN);
         }
     }

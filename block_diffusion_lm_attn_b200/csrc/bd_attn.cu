@@ -22,6 +22,7 @@
 #include "attn_tc_persist.cuh"
 #include "attn_tc_pair.cuh"
 #include "bd_common.cuh"
+#include "cache_ops.cuh"
 
 namespace {
 
@@ -93,7 +94,7 @@ struct DecodePlan {
 bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
                  DecodePlan &pl)
 {
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap < b ||
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0 ||
         Hq % Hkv != 0)
         return false;
     const long long rows = (long long)(Hq / Hkv) * b;
@@ -266,9 +267,10 @@ bd_status decode_validate(const void *q_blk, const void *k_cache,
         return BD_ERR_INVALID_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
         return BD_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0 || S_cap < b)
+    if (mode < 0 || mode > 2)
         return BD_ERR_INVALID_ARG;
-    if (mode != 0 && mode != 1)
+    // modes 0 and 1 read the block's own keys after the prefix
+    if (Hq % Hkv != 0 || (mode != 2 && S_cap < b))
         return BD_ERR_INVALID_ARG;
     if (!supported_d(d))
         return BD_ERR_UNSUPPORTED;
@@ -471,6 +473,110 @@ bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
     return decode_launch(q_blk, k_cache, v_cache, cache_len, out, lse, B, Hq,
                          Hkv, b, d, intra_block_mode, stream, S_cap, workspace,
                          pl);
+}
+
+bd_status bd_spec_accept(const int32_t *draft, const int32_t *target,
+                         int32_t *n_accept, int B, int b, cudaStream_t stream)
+{
+    if (!draft || !target || !n_accept || B <= 0 || b <= 0)
+        return BD_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(draft) | reinterpret_cast<uintptr_t>(target) |
+         reinterpret_cast<uintptr_t>(n_accept)) & 3u)
+        return BD_ERR_INVALID_ARG;
+    bd::bd_spec_accept_kernel<<<(B + 7) / 8, 256, 0, stream>>>(draft, target,
+                                                               n_accept, B, b);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+bd_status bd_cache_append(void *k_cache, void *v_cache, int32_t *cache_len,
+                          const void *k_new, const void *v_new,
+                          const int32_t *n_new, int B, int Hkv, int b, int d,
+                          int S_cap, cudaStream_t stream)
+{
+    if (!k_cache || !v_cache || !cache_len || !n_new || (!k_new != !v_new))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hkv <= 0 || b <= 0 || d <= 0 || S_cap <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || (k_new && !aligned16(k_new)) ||
+        (v_new && !aligned16(v_new)) ||
+        ((reinterpret_cast<uintptr_t>(cache_len) | reinterpret_cast<uintptr_t>(n_new)) & 3u))
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    bd::bd_cache_append_kernel<<<B, 512, 0, stream>>>(
+        static_cast<bf16 *>(k_cache), static_cast<bf16 *>(v_cache), cache_len,
+        static_cast<const bf16 *>(k_new), static_cast<const bf16 *>(v_new), n_new, Hkv, b,
+        d, S_cap);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+bd_status bd_cache_crop(int32_t *cache_len, int B, int max_len,
+                        cudaStream_t stream)
+{
+    if (!cache_len || B <= 0 || max_len < 0 ||
+        (reinterpret_cast<uintptr_t>(cache_len) & 3u))
+        return BD_ERR_INVALID_ARG;
+    bd::bd_cache_crop_kernel<<<(B + 255) / 256, 256, 0, stream>>>(cache_len, B, max_len);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+size_t bd_sprint_workspace_bytes(int B, int S_cap)
+{
+    if (B <= 0 || S_cap <= 0)
+        return 0;
+    return 2 * round256((size_t)B * S_cap * sizeof(double));
+}
+
+bd_status bd_sprint_prune(const void *k_cache, const void *v_cache,
+                          const int32_t *cache_len, const float *conf,
+                          const uint8_t *modality, float alpha,
+                          float keep_text, float keep_image, void *k_out,
+                          void *v_out, int32_t *kept, int32_t *new_len,
+                          double *score, int B, int Hkv, int d, int S_cap,
+                          cudaStream_t stream, void *workspace,
+                          size_t workspace_bytes)
+{
+    if (!k_cache || !v_cache || !cache_len || !conf || !modality || !k_out ||
+        !v_out || !kept || !new_len || !workspace)
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hkv <= 0 || d <= 0 || S_cap <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (!(alpha >= 0.f && alpha <= 1.f) || !(keep_text >= 0.f && keep_text <= 1.f) ||
+        !(keep_image >= 0.f && keep_image <= 1.f))
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(k_out) ||
+        !aligned16(v_out) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        ((reinterpret_cast<uintptr_t>(cache_len) | reinterpret_cast<uintptr_t>(conf) |
+          reinterpret_cast<uintptr_t>(kept) | reinterpret_cast<uintptr_t>(new_len)) & 3u) ||
+        (score && (reinterpret_cast<uintptr_t>(score) & 7u)))
+        return BD_ERR_INVALID_ARG;
+    if (k_out == k_cache || v_out == v_cache || k_out == v_cache || v_out == k_cache)
+        return BD_ERR_INVALID_ARG;
+    if (workspace_bytes < bd_sprint_workspace_bytes(B, S_cap))
+        return BD_ERR_INVALID_ARG;
+    if (!supported_d(d))
+        return BD_ERR_UNSUPPORTED;
+    // the select kernel holds at most 64 positions per thread
+    if (S_cap > 64 * bd::kSelThreads || B > 65535)
+        return BD_ERR_UNSUPPORTED;
+    double *norm = static_cast<double *>(workspace);
+    double *sc = score ? score
+                       : reinterpret_cast<double *>(static_cast<char *>(workspace) +
+                                                    round256((size_t)B * S_cap * sizeof(double)));
+    dim3 gn((S_cap + 7) / 8, B);
+    bd::bd_sprint_norm_kernel<<<gn, 256, 0, stream>>>(static_cast<const bf16 *>(k_cache),
+                                                      cache_len, norm, Hkv, d, S_cap);
+    if (cudaGetLastError() != cudaSuccess)
+        return BD_ERR_CUDA;
+    bd::bd_sprint_select_kernel<<<B, bd::kSelThreads, 0, stream>>>(
+        norm, cache_len, conf, modality, (double)alpha, (double)keep_text, (double)keep_image,
+        sc, kept, new_len, S_cap);
+    if (cudaGetLastError() != cudaSuccess)
+        return BD_ERR_CUDA;
+    bd::bd_sprint_compact_kernel<<<gn, 256, 0, stream>>>(
+        static_cast<const bf16 *>(k_cache), static_cast<const bf16 *>(v_cache), kept, new_len,
+        static_cast<bf16 *>(k_out), static_cast<bf16 *>(v_out), Hkv, d, S_cap);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
 }
 
 bd_status bd_attn_debug_inject_fault(int kind)

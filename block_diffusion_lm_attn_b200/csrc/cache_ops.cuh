@@ -1,0 +1,369 @@
+// KV-cache kernels of block decoding (sm_100a): accepting a speculated
+// block, appending it to the cache, cropping the cache, and sparse prefix
+// retention (SPRINT).
+//
+//  - Speculative accept / append / crop: "Nemotron-Labs-Diffusion-8B-Base 3x
+//    decoding speed-up", section 2 "Linear Speculative Decoding" (draft a
+//    block with bidirectional attention, validate it with causal attention,
+//    accept the longest matching prefix, update the KV cache) and section
+//    "KV cache strategy" (crop the cache to a maximum length).
+//  - Sparse prefix retention: "LLaDA2.0-Uni", section "SPRINT: training-free
+//    inference acceleration", paragraph "Sparse Prefix Retention": once per
+//    block, score every prefix position by s_i = alpha * I_i + (1 - alpha) *
+//    c_i, I_i = |k_i|_2 / mean_j |k_j|_2, and keep each modality's best
+//    fraction (images 0.8, text 1.0 on the page).
+//
+// Layouts as in the attention kernels: caches [B, Hkv, S_cap, d] bf16,
+// cache_len [B] int32 on the device.  All of it is HBM- or latency-bound:
+// 16-byte vector copies, fp64 only for the SPRINT scores (so the kept set
+// is decided in double precision).
+#pragma once
+
+#include "bd_common.cuh"
+
+namespace bd {
+
+// ---------------------------------------------------------------------------
+// speculative decoding: accepted length, append, crop
+
+// n_accept[i] = length of the longest prefix of block positions j on which
+// draft[i][j] == target[i][j].  One warp per sequence.
+__global__ void __launch_bounds__(256)
+    bd_spec_accept_kernel(const int32_t *draft, const int32_t *target,
+                          int32_t *n_accept, int B, int b)
+{
+    const int i = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (i >= B)
+        return;
+    const int32_t *dr = draft + (size_t)i * b;
+    const int32_t *tg = target + (size_t)i * b;
+    int n = b;
+    for (int j0 = 0; j0 < b; j0 += 32) {
+        const int j = j0 + lane;
+        const bool differ = j < b && dr[j] != tg[j];
+        const unsigned m = __ballot_sync(0xffffffffu, differ);
+        if (m) {
+            n = j0 + __ffs(m) - 1;
+            break;
+        }
+    }
+    if (lane == 0)
+        n_accept[i] = n;
+}
+
+// Appends rows 0 .. n_new[i]-1 of the block K/V ([B, Hkv, b, d]; NULL: the
+// rows already sit at cache positions cache_len[i] ..) and advances
+// cache_len[i].  One CTA per sequence, so the length is updated after every
+// copy of that sequence has read it.  An out-of-range n_new or length leaves
+// the sequence untouched and records DEV_BAD_CACHE_LEN.
+__global__ void __launch_bounds__(512)
+    bd_cache_append_kernel(bf16 *k_cache, bf16 *v_cache, int32_t *cache_len,
+                           const bf16 *k_new, const bf16 *v_new,
+                           const int32_t *n_new, int Hkv, int b, int d,
+                           int S_cap)
+{
+    const int i = blockIdx.x;
+    const int len = cache_len[i];
+    const int n = n_new[i];
+    if (n < 0 || n > b || len < 0 || (long long)len + n > S_cap) {
+        if (threadIdx.x == 0)
+            raise_device_code(DEV_BAD_CACHE_LEN);
+        return;
+    }
+    if (k_new != nullptr) {
+        const int vec_per_row = d / 8; // 16-byte vectors
+        const long long total = (long long)Hkv * n * vec_per_row;
+        for (long long e = threadIdx.x; e < total; e += blockDim.x) {
+            const int c = (int)(e % vec_per_row);
+            const long long rr = e / vec_per_row;
+            const int r = (int)(rr % n), h = (int)(rr / n);
+            const size_t src = (((size_t)i * Hkv + h) * b + r) * d + (size_t)c * 8;
+            const size_t dst = (((size_t)i * Hkv + h) * S_cap + len + r) * d + (size_t)c * 8;
+            reinterpret_cast<uint4 *>(k_cache + dst)[0] =
+                reinterpret_cast<const uint4 *>(k_new + src)[0];
+            reinterpret_cast<uint4 *>(v_cache + dst)[0] =
+                reinterpret_cast<const uint4 *>(v_new + src)[0];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        cache_len[i] = len + n;
+}
+
+// cache_len[i] = min(cache_len[i], max_len).
+__global__ void __launch_bounds__(256)
+    bd_cache_crop_kernel(int32_t *cache_len, int B, int max_len)
+{
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < B)
+        cache_len[i] = min(cache_len[i], max_len);
+}
+
+// ---------------------------------------------------------------------------
+// sparse prefix retention
+
+// |k_p|_2 over all kv-heads and dims of position p, for p < cache_len[i]:
+// norm[i][p] in fp64.  One warp per position; lane l reads 16-byte pieces
+// of the position's Hkv rows (two rows per warp load, each row contiguous).
+__global__ void __launch_bounds__(256)
+    bd_sprint_norm_kernel(const bf16 *k_cache, const int32_t *cache_len,
+                          double *norm, int Hkv, int d, int S_cap)
+{
+    const int i = blockIdx.y;
+    const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int len = cache_len[i];
+    if (p >= S_cap || p >= len || len > S_cap)
+        return;
+    const int vec_per_row = d / 8;
+    const int nvec = Hkv * vec_per_row;
+    double ss = 0.0;
+    for (int e = lane; e < nvec; e += 32) {
+        const int h = e / vec_per_row, c = e % vec_per_row;
+        const uint4 x = *reinterpret_cast<const uint4 *>(
+            k_cache + (((size_t)i * Hkv + h) * S_cap + p) * d + (size_t)c * 8);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const double lo = (double)__uint_as_float(w[t] << 16);
+            const double hi = (double)__uint_as_float(w[t] & 0xffff0000u);
+            ss = fma(lo, lo, ss);
+            ss = fma(hi, hi, ss);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0)
+        norm[(size_t)i * S_cap + p] = sqrt(ss);
+}
+
+constexpr int kSelThreads = 1024;
+
+// Order-preserving map of a double onto uint64 (larger value -> larger key).
+__device__ __forceinline__ unsigned long long dkey(double x)
+{
+    const unsigned long long u = (unsigned long long)__double_as_longlong(x);
+    return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
+
+template <typename T> __device__ T block_sum(T v, T *red)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __syncthreads();
+    if (lane == 0)
+        red[w] = v;
+    __syncthreads();
+    T tot = 0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k)
+        tot += red[k];
+    return tot;
+}
+
+// Exclusive prefix sum of one int per thread over the block (in thread
+// order); returns the thread's offset and writes the total.
+__device__ int block_scan_excl(int v, int *red, int &total)
+{
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o)
+            x += y;
+    }
+    __syncthreads();
+    if (lane == 31)
+        red[w] = x;
+    __syncthreads();
+    int base = 0, tot = 0;
+    for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+        if (k < w)
+            base += red[k];
+        tot += red[k];
+    }
+    total = tot;
+    return base + x - v;
+}
+
+// Scores, per-modality selection and the kept list of one sequence per CTA.
+//   score[i][p] = alpha * norm_p / mean + (1 - alpha) * conf[i][p] (fp64),
+//   per modality m (0 text, else image) with n_m prefix positions keep the
+//   floor(r_m n_m + 1/2) best (higher score, then lower position),
+//   kept[i][0 .. new_len-1] = kept positions in increasing order, then -1.
+// The threshold of each modality is found by an 8-pass radix select (8 bits
+// per pass) over the score keys; positions are visited in contiguous
+// per-thread runs so that the final scan keeps position order.
+__global__ void __launch_bounds__(kSelThreads)
+    bd_sprint_select_kernel(const double *norm, const int32_t *cache_len,
+                            const float *conf, const uint8_t *modality,
+                            double alpha, double keep_text, double keep_image,
+                            double *score, int32_t *kept, int32_t *new_len,
+                            int S_cap)
+{
+    __shared__ double red_d[32];
+    __shared__ int red_i[32];
+    __shared__ unsigned int hist[256];
+    __shared__ unsigned long long s_prefix;
+    __shared__ int s_need;
+    const int i = blockIdx.x;
+    const int len = cache_len[i];
+    const int tid = threadIdx.x;
+    const size_t row = (size_t)i * S_cap;
+    if (len < 0 || len > S_cap) {
+        if (tid == 0) {
+            raise_device_code(DEV_BAD_CACHE_LEN);
+            new_len[i] = 0;
+        }
+        for (int p = tid; p < S_cap; p += blockDim.x)
+            kept[row + p] = -1;
+        return;
+    }
+    // this thread's contiguous run of positions [p0, p1)
+    const int per = (len + blockDim.x - 1) / blockDim.x;
+    const int p0 = min(len, tid * per), p1 = min(len, p0 + per);
+
+    double part = 0.0;
+    for (int p = p0; p < p1; ++p)
+        part += norm[row + p];
+    const double mean = block_sum(part, red_d) / (double)max(len, 1);
+    for (int p = p0; p < p1; ++p) {
+        // separate roundings, no fused multiply-add: the same arithmetic as
+        // the plain definition, so equal inputs give equal scores
+        const double inorm = mean > 0.0 ? __ddiv_rn(norm[row + p], mean) : 0.0;
+        score[row + p] = __dadd_rn(__dmul_rn(alpha, inorm),
+                                   __dmul_rn(__dadd_rn(1.0, -alpha), (double)conf[row + p]));
+    }
+    __syncthreads();
+
+    // kept flags live in the kept row itself until the final compaction:
+    // 1 = kept, 0 = dropped
+    for (int m = 0; m < 2; ++m) {
+        int cnt = 0;
+        for (int p = p0; p < p1; ++p)
+            cnt += ((modality[row + p] != 0) == m);
+        const int n_m = block_sum(cnt, red_i);
+        const double r = m == 0 ? keep_text : keep_image;
+        long long want = (long long)floor(r * (double)n_m + 0.5);
+        want = max(0LL, min(want, (long long)n_m));
+        // radix select of the want-th largest key among this modality
+        if (tid == 0) {
+            s_prefix = 0;
+            s_need = (int)want; // rank still to find inside the prefix
+        }
+        __syncthreads();
+        if (want > 0) {
+            for (int pass = 0; pass < 8; ++pass) {
+                const int shift = 56 - 8 * pass;
+                for (int k = tid; k < 256; k += blockDim.x)
+                    hist[k] = 0;
+                __syncthreads();
+                const unsigned long long pre = s_prefix;
+                const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+                for (int p = p0; p < p1; ++p) {
+                    if ((modality[row + p] != 0) != m)
+                        continue;
+                    const unsigned long long key = dkey(score[row + p]);
+                    if ((key & hmask) == pre)
+                        atomicAdd(&hist[(key >> shift) & 255], 1u);
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    int need = s_need;
+                    int dgt = 255;
+                    for (; dgt > 0; --dgt) {
+                        if ((int)hist[dgt] >= need)
+                            break;
+                        need -= (int)hist[dgt];
+                    }
+                    s_prefix = pre | ((unsigned long long)dgt << shift);
+                    s_need = need;
+                }
+                __syncthreads();
+            }
+        }
+        // keys above the threshold are kept; of the keys equal to it, the
+        // s_need lowest positions
+        const unsigned long long thr = s_prefix;
+        const int need_eq = want > 0 ? s_need : 0;
+        int eq = 0;
+        for (int p = p0; p < p1; ++p)
+            if ((modality[row + p] != 0) == m && want > 0 &&
+                dkey(score[row + p]) == thr)
+                ++eq;
+        int tot_eq;
+        int before = block_scan_excl(eq, red_i, tot_eq);
+        for (int p = p0; p < p1; ++p) {
+            if ((modality[row + p] != 0) != m)
+                continue;
+            int keep = 0;
+            if (want > 0) {
+                const unsigned long long key = dkey(score[row + p]);
+                if (key > thr)
+                    keep = 1;
+                else if (key == thr)
+                    keep = (before++ < need_eq);
+            }
+            kept[row + p] = keep;
+        }
+        __syncthreads();
+    }
+
+    // stable compaction of the kept positions
+    int mine = 0;
+    for (int p = p0; p < p1; ++p)
+        mine += kept[row + p];
+    int total;
+    int dst = block_scan_excl(mine, red_i, total);
+    // read the flags of this thread's run before any thread overwrites them
+    // with positions: a thread's destinations can reach into the runs of
+    // threads before it only, whose flags those threads already hold
+    int flags[64];
+    int nf = 0;
+    for (int p = p0; p < p1 && nf < 64; ++p)
+        flags[nf++] = kept[row + p];
+    __syncthreads();
+    if (per <= 64) {
+        for (int p = p0, k = 0; p < p1; ++p, ++k)
+            if (flags[k])
+                kept[row + dst++] = p;
+    }
+    __syncthreads();
+    for (int p = total + tid; p < S_cap; p += blockDim.x)
+        kept[row + p] = -1;
+    if (tid == 0)
+        new_len[i] = total;
+}
+
+// k_out/v_out rows 0 .. new_len[i]-1 = k_cache/v_cache rows kept[i][0 ..]
+// for every kv-head.  Grid (S_cap / 8 tiles, B); one warp per destination
+// row of all heads, 16-byte vectors.
+__global__ void __launch_bounds__(256)
+    bd_sprint_compact_kernel(const bf16 *k_cache, const bf16 *v_cache,
+                             const int32_t *kept, const int32_t *new_len,
+                             bf16 *k_out, bf16 *v_out, int Hkv, int d,
+                             int S_cap)
+{
+    const int i = blockIdx.y;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (t >= new_len[i])
+        return;
+    const int src = kept[(size_t)i * S_cap + t];
+    const int vec_per_row = d / 8;
+    const int nvec = Hkv * vec_per_row;
+    for (int e = lane; e < nvec; e += 32) {
+        const int h = e / vec_per_row, c = e % vec_per_row;
+        const size_t hb = ((size_t)i * Hkv + h) * S_cap;
+        const size_t so = (hb + src) * d + (size_t)c * 8;
+        const size_t dof = (hb + t) * d + (size_t)c * 8;
+        reinterpret_cast<uint4 *>(k_out + dof)[0] = reinterpret_cast<const uint4 *>(k_cache + so)[0];
+        reinterpret_cast<uint4 *>(v_out + dof)[0] = reinterpret_cast<const uint4 *>(v_cache + so)[0];
+    }
+}
+
+} // namespace bd

@@ -177,6 +177,123 @@ BD_API bd_status bd_attn_decode_noalloc(const void *q_blk, const void *k_cache,
                                         int b, int d, int intra_block_mode,
                                         struct CUstream_st *stream, int S_cap);
 
+/*
+ * Speculative decoding: accepted prefix length.
+ *
+ * Defines: "Nemotron-Labs-Diffusion-8B-Base 3x decoding speed-up", section 2
+ * "Linear Speculative Decoding": a block drafted with bidirectional attention
+ * is validated with causal attention and its longest matching prefix is
+ * accepted.
+ *
+ *   draft, target  [B, b] int32 tokens, DEVICE memory (read): the drafted
+ *                  block and the verifier's token for each block position
+ *   n_accept       [B] int32, DEVICE memory (written): the length of the
+ *                  longest prefix j = 0 .. n-1 with draft[i][j] == target[i][j]
+ *
+ * Errors: BD_ERR_INVALID_ARG for a null or non-4-byte-aligned pointer or a
+ * size <= 0; BD_ERR_CUDA if the launch fails.
+ */
+BD_API bd_status bd_spec_accept(const int32_t *draft, const int32_t *target,
+                                int32_t *n_accept, int B, int b,
+                                struct CUstream_st *stream);
+
+/*
+ * Append accepted rows to the KV cache and advance its length, on the device.
+ *
+ * Defines: the "update the KV cache" step of linear speculative decoding,
+ * "Nemotron-Labs-Diffusion-8B-Base 3x decoding speed-up", section 2.
+ *
+ *   k_cache, v_cache  [B, Hkv, S_cap, d] bf16 (read and written in place)
+ *   cache_len         [B] int32, DEVICE memory (read, then advanced by
+ *                     n_new[i])
+ *   k_new, v_new      [B, Hkv, b, d] bf16 (read): the block's K/V; rows
+ *                     0 .. n_new[i]-1 are copied to cache positions
+ *                     cache_len[i] .. cache_len[i]+n_new[i]-1.  Both NULL:
+ *                     the rows are already there (the usual case: the block's
+ *                     K/V were written at the cache tail before the causal
+ *                     verification), so only the length advances.
+ *   n_new             [B] int32, DEVICE memory (read), e.g. from
+ *                     bd_spec_accept
+ *
+ * Nothing is allocated; the call can be captured in a CUDA graph.  A
+ * sequence with n_new[i] outside [0, b] or cache_len[i] + n_new[i] > S_cap is
+ * left untouched and the device status word records BD_ERR_DEVICE_TIMEOUT.
+ * Errors: BD_ERR_INVALID_ARG for a null pointer (k_new and v_new must be both
+ * NULL or both set), a misaligned pointer or a size <= 0;
+ * BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA if the launch
+ * fails.
+ */
+BD_API bd_status bd_cache_append(void *k_cache, void *v_cache, int32_t *cache_len,
+                                 const void *k_new, const void *v_new,
+                                 const int32_t *n_new, int B, int Hkv, int b,
+                                 int d, int S_cap, struct CUstream_st *stream);
+
+/*
+ * Crop the KV cache to at most max_len positions: cache_len[i] =
+ * min(cache_len[i], max_len), on the device (the cache rows stay where they
+ * are).  Defines: "Nemotron-Labs-Diffusion-8B-Base 3x decoding speed-up",
+ * section "KV cache strategy" (the cache is cropped to a maximum length
+ * during generation).  cache_len: [B] int32 in DEVICE memory.
+ * Errors: BD_ERR_INVALID_ARG for a null or misaligned pointer, B <= 0 or
+ * max_len < 0; BD_ERR_CUDA if the launch fails.
+ */
+BD_API bd_status bd_cache_crop(int32_t *cache_len, int B, int max_len,
+                               struct CUstream_st *stream);
+
+/*
+ * Sparse prefix retention (SPRINT): prune the cached prefix once at the start
+ * of a block.
+ *
+ * Defines: "LLaDA2.0-Uni" (discuss.pytorch.kr), section "SPRINT: training-free
+ * inference acceleration", paragraph "Sparse Prefix Retention".  Each prefix
+ * position p < cache_len[i] gets the score
+ *     s_p = alpha * I_p + (1 - alpha) * conf[i][p],
+ *     I_p = |k_p|_2 / mean over the prefix of |k_j|_2,
+ * where |k_p|_2 is the norm of position p's key over all kv-heads and dims
+ * of this cache (0 for all p if that mean is 0), and conf is the caller's
+ * top-1 softmax confidence.  Each modality (modality[i][p] == 0: text, else
+ * image) with n prefix positions keeps floor(r * n + 1/2) of them, r =
+ * keep_text or keep_image: those with the highest score, ties to the lower
+ * position.  The page uses alpha = 0.5, keep_image = 0.8, keep_text = 1.0.
+ * The kept positions, in their original order, become the new prefix.
+ * Scores are computed in double precision.
+ *
+ *   k_cache, v_cache  [B, Hkv, S_cap, d] bf16 (read)
+ *   cache_len         [B] int32, DEVICE (read)
+ *   conf              [B, S_cap] fp32, DEVICE (read; entries < cache_len[i])
+ *   modality          [B, S_cap] uint8, DEVICE (read; entries < cache_len[i])
+ *   k_out, v_out      [B, Hkv, S_cap, d] bf16 (written: rows 0 ..
+ *                     new_len[i]-1 are the kept rows; later rows untouched).
+ *                     Must not overlap the input caches.
+ *   kept              [B, S_cap] int32, DEVICE (written: kept positions in
+ *                     increasing order, then -1)
+ *   new_len           [B] int32, DEVICE (written; the prefix length to pass to
+ *                     bd_attn_decode as cache_len afterwards)
+ *   score             [B, S_cap] fp64, DEVICE (written for p < cache_len[i])
+ *                     or NULL
+ *   workspace         DEVICE scratch of bd_sprint_workspace_bytes(B, S_cap)
+ *                     bytes, 256-byte aligned
+ *
+ * Errors: BD_ERR_INVALID_ARG for a null (other than score) or misaligned
+ * pointer, a size <= 0, alpha or a keep ratio outside [0, 1], aliasing
+ * outputs, or a short workspace; BD_ERR_UNSUPPORTED for d not in {32, 64,
+ * 128} or S_cap > 65536; BD_ERR_CUDA if a launch fails.  A cache_len[i]
+ * outside [0, S_cap] gives new_len[i] = 0 and records BD_ERR_DEVICE_TIMEOUT
+ * in the device status word.
+ */
+BD_API bd_status bd_sprint_prune(const void *k_cache, const void *v_cache,
+                                 const int32_t *cache_len, const float *conf,
+                                 const uint8_t *modality, float alpha,
+                                 float keep_text, float keep_image,
+                                 void *k_out, void *v_out, int32_t *kept,
+                                 int32_t *new_len, double *score, int B,
+                                 int Hkv, int d, int S_cap,
+                                 struct CUstream_st *stream, void *workspace,
+                                 size_t workspace_bytes);
+
+/* Bytes of scratch bd_sprint_prune needs (0 on bad sizes).  Host only. */
+BD_API size_t bd_sprint_workspace_bytes(int B, int S_cap);
+
 /* Bytes of scratch bd_attn_decode needs for these sizes (0 on bad sizes).
  * Pure host arithmetic; needs no GPU. */
 BD_API size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int d,

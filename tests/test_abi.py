@@ -44,7 +44,9 @@ def test_workspace_bytes(lib):
     assert bd.bd_attn_decode_workspace_bytes(16, 32, 8, 32, 128, 8224) > 0
     assert bd.bd_attn_decode_workspace_bytes(0, 32, 8, 32, 128, 8224) == 0
     assert bd.bd_attn_decode_workspace_bytes(1, 6, 4, 32, 128, 64) == 0
-    assert bd.bd_attn_decode_workspace_bytes(1, 4, 4, 32, 128, 16) == 0
+    assert bd.bd_attn_decode_workspace_bytes(1, 4, 4, 32, 128, 0) == 0
+    # a cache shorter than the block is valid for cross-attention (mode 2)
+    assert bd.bd_attn_decode_workspace_bytes(1, 4, 4, 32, 128, 16) > 0
     w = bd.bd_attn_decode_workspace_bytes(16, 32, 8, 32, 128, 8224)
     assert w % 256 == 0
 
@@ -91,7 +93,8 @@ def dec_args(**kw):
     (dict(cache_len=A + 2), bd.BD_ERR_INVALID_ARG),
     (dict(Hq=3), bd.BD_ERR_INVALID_ARG),
     (dict(S_cap=4), bd.BD_ERR_INVALID_ARG),
-    (dict(intra_block_mode=2), bd.BD_ERR_INVALID_ARG),
+    (dict(intra_block_mode=3), bd.BD_ERR_INVALID_ARG),
+    (dict(intra_block_mode=-1), bd.BD_ERR_INVALID_ARG),
     (dict(b=0), bd.BD_ERR_INVALID_ARG),
     (dict(workspace_bytes=16), bd.BD_ERR_INVALID_ARG),
     (dict(workspace=A + 16), bd.BD_ERR_INVALID_ARG),
@@ -119,3 +122,37 @@ def test_grid_hook_rejects_out_of_range(lib):
     assert bd.bd_attn_debug_set_grid(-1) == bd.BD_ERR_INVALID_ARG
     assert bd.bd_attn_debug_set_grid(149) == bd.BD_ERR_INVALID_ARG
     assert bd.bd_attn_debug_set_grid(0) == bd.BD_OK
+
+
+def test_cache_and_sprint_reject_bad_arguments(lib):
+    I = bd.BD_ERR_INVALID_ARG
+    U = bd.BD_ERR_UNSUPPORTED
+    assert bd.bd_spec_accept(None, A, A, 4, 8, None) == I
+    assert bd.bd_spec_accept(A, A + 2, A, 4, 8, None) == I
+    assert bd.bd_spec_accept(A, A, A, 0, 8, None) == I
+    # k_new and v_new must be both given or both NULL
+    assert bd.bd_cache_append(A, A, A, A, None, A, 2, 2, 4, 64, 32, None) == I
+    assert bd.bd_cache_append(A, A + 8, A, None, None, A, 2, 2, 4, 64, 32, None) == I
+    assert bd.bd_cache_append(A, A, A, None, None, A, 2, 2, 4, 80, 32, None) == U
+    assert bd.bd_cache_crop(A, 4, -1, None) == I
+    assert bd.bd_cache_crop(None, 4, 3, None) == I
+    ws = bd.bd_sprint_workspace_bytes(2, 64)
+    assert ws > 0 and ws % 256 == 0 and bd.bd_sprint_workspace_bytes(0, 64) == 0
+
+    def sp(**kw):
+        a = dict(k_cache=A, v_cache=A + 4096, cache_len=A, conf=A, modality=A,
+                 alpha=0.5, keep_text=1.0, keep_image=0.8, k_out=A + 8192,
+                 v_out=A + 12288, kept=A, new_len=A, score=None, B=2, Hkv=2,
+                 d=64, S_cap=64, stream=None, workspace=A, workspace_bytes=ws)
+        a.update(kw)
+        return bd.bd_sprint_prune(**a)
+    assert sp(conf=None) == I
+    assert sp(alpha=1.5) == I
+    assert sp(keep_image=-0.1) == I
+    assert sp(keep_text=float("nan")) == I
+    assert sp(k_out=A) == I                  # output aliases the input cache
+    assert sp(workspace_bytes=ws - 1) == I
+    assert sp(workspace=A + 16) == I
+    assert sp(score=A + 4) == I
+    assert sp(d=48) == U
+    assert sp(S_cap=65537, workspace_bytes=1 << 40) == U
