@@ -354,6 +354,11 @@ __global__ void __launch_bounds__(256)
     if (t >= new_len[i])
         return;
     const int src = kept[(size_t)i * S_cap + t];
+    if (src < 0 || src >= S_cap) { // cannot happen after the select kernel
+        if (lane == 0)
+            raise_device_code(DEV_BAD_CACHE_LEN);
+        return;
+    }
     const int vec_per_row = d / 8;
     const int nvec = Hkv * vec_per_row;
     for (int e = lane; e < nvec; e += 32) {

@@ -105,7 +105,14 @@ BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *
  * prefix only.  Block row j of sequence i sees cache positions
  * 0 .. cache_len[i]-1 and block positions cache_len[i]+j' for every j' < b
  * (intra_block_mode 0, bidirectional denoise) or every j' <= j
- * (intra_block_mode 1, causal verify).  Softmax scale is 1/sqrt(d).
+ * (intra_block_mode 1, causal verify).  intra_block_mode 2 is cross-attention
+ * only: the b rows are the canvas of an encoder-decoder model and see the
+ * encoder's cache positions 0 .. cache_len[i]-1 and nothing of themselves
+ * ("DiffusionGemma" pipeline page of the diffusers docs, introduction and
+ * pipeline class description: a bidirectional decoder cross-attends to the
+ * KV cache a causal encoder wrote, to denoise a canvas of canvas_length
+ * tokens); with cache_len[i] = 0 such rows see nothing and get out = 0,
+ * lse = -inf.  Softmax scale is 1/sqrt(d).
  *
  *   q_blk            [B, Hq, b, d]        bf16 (read)
  *   k_cache, v_cache [B, Hkv, S_cap, d]   bf16 (read; rows beyond
@@ -115,7 +122,7 @@ BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *
  *                    a CUDA graph)
  *   out              [B, Hq, b, d]        bf16 (written)
  *   lse              [B, Hq, b]           fp32 (written)
- *   S_cap            row capacity of the caches (>= b)
+ *   S_cap            row capacity of the caches (>= b in modes 0 and 1)
  *   workspace        device scratch of at least
  *                    bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap)
  *                    bytes, 256-byte aligned, used for the split-KV partial
@@ -125,12 +132,13 @@ BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *
  *                    not be inside a stream capture).
  *
  * Errors: BD_ERR_INVALID_ARG for a null or misaligned pointer, any size <= 0,
- * Hq % Hkv != 0, S_cap < b, intra_block_mode not 0/1, or a workspace smaller
- * than required; BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA
- * if the launch (or the internal workspace allocation) fails.  A cache_len[i]
- * outside [0, S_cap - b] is caught on the device: that sequence's rows are
- * written as NaN with lse NaN, and the device status word (see
- * bd_attn_get_device_status) records BD_ERR_DEVICE_TIMEOUT.
+ * Hq % Hkv != 0, S_cap < b in modes 0 and 1, intra_block_mode not 0/1/2, or
+ * a workspace smaller than required; BD_ERR_UNSUPPORTED for d not in {32,
+ * 64, 128}; BD_ERR_CUDA if the launch (or the internal workspace allocation)
+ * fails.  A cache_len[i] outside [0, S_cap - b] (modes 0 and 1) or [0, S_cap]
+ * (mode 2) is caught on the device: that sequence's rows are written as NaN
+ * with lse NaN, and the device status word (see bd_attn_get_device_status)
+ * records BD_ERR_DEVICE_TIMEOUT.
  */
 BD_API bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
                          const void *v_cache, const int32_t *cache_len,
