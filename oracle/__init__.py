@@ -69,7 +69,7 @@ def _bind(lib):
     lib.bdo_fwd_mask.argtypes = [ctypes.c_int, ctypes.c_int, _u8p]
     lib.bdo_sprint_select.restype = ctypes.c_int
     lib.bdo_sprint_select.argtypes = [_u16p, _i32p, _f32p, _u8p] + [
-        ctypes.c_int] * 4 + [ctypes.c_double] * 3 + [_f64p, _i32p, _i32p]
+        ctypes.c_int] * 4 + [ctypes.c_float] * 3 + [_f64p, _i32p, _i32p]
     lib.bdo_combine.restype = None
     lib.bdo_combine.argtypes = [ctypes.c_int, ctypes.c_int, _f64p, _f64p,
                                 _f64p, _f64p]
@@ -225,7 +225,8 @@ def sprint_select(k_cache, cache_len, conf, modality, alpha=0.5,
     k_cache [B,Hkv,S_cap,d] bf16; cache_len [B]; conf [B,S_cap] fp32 top-1
     confidences; modality [B,S_cap] uint8 (0 text, else image).  Returns
     (score [B,S_cap] fp64, kept [B,S_cap] int32 -- kept positions in order,
-    then -1 --, new_len [B] int32)."""
+    then -1 --, new_len [B] int32).  alpha and the keep ratios are rounded
+    to single precision first, as the library's interface takes them."""
     lib = lib or load()
     B, Hkv, S_cap, d = k_cache.shape
     kb = _bits(k_cache)

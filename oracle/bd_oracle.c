@@ -380,8 +380,9 @@ void bdo_combine(int nparts, int d, const double *o_s, const double *lse_s,
  *    so |k_i|_2 = sqrt(sum over heads h and dims t of k[h][i][t]^2);
  *  - the mean in I_i runs over the prefix positions 0..cache_len-1 (the L of
  *    the page's formula); if it is 0 (an all-zero prefix) every I_i is 0;
- *  - modality 0 is text, any other value image; a modality with n prefix
- *    positions keeps floor(r * n + 1/2) of them (r widened to double),
+ *  - alpha and the keep ratios r are single-precision numbers; modality 0
+ *    is text, any other value image; a modality with n prefix positions
+ *    keeps floor(r * n + 1/2) of them (r widened to double),
  *    clamped to [0, n]: the best scores, ties broken by the lower position;
  *  - the kept positions stay in their original order (stable compaction)
  *    and become the new prefix.
@@ -411,10 +412,12 @@ static int bdo_scored_cmp(const void *a, const void *b)
  * -1, and new_len: [B], their number.  Returns 0, or -1 on a bad argument. */
 int bdo_sprint_select(const uint16_t *k_cache, const int32_t *cache_len,
                       const float *conf, const uint8_t *modality, int B,
-                      int Hkv, int d, int S_cap, double alpha,
-                      double keep_text, double keep_image, double *score,
+                      int Hkv, int d, int S_cap, float alpha_f,
+                      float keep_text_f, float keep_image_f, double *score,
                       int32_t *kept, int32_t *new_len)
 {
+    /* alpha and the keep ratios are single-precision inputs, widened */
+    const double alpha = alpha_f, keep_text = keep_text_f, keep_image = keep_image_f;
     if (B <= 0 || Hkv <= 0 || d <= 0 || S_cap <= 0)
         return -1;
     if (!(alpha >= 0.0 && alpha <= 1.0) || !(keep_text >= 0.0 && keep_text <= 1.0) ||

@@ -144,6 +144,7 @@ def pin_sprint_alpha_limits_are_sorts(lib):
                     np.testing.assert_allclose(score[i, :n], sc, rtol=1e-13)
                 want = []
                 for m, r in ((0, kt), (1, ki)):
+                    r = float(np.float32(r))  # the interface's precision
                     pos = [p for p in range(n) if (mod[i, p] != 0) == m]
                     cnt = int(math.floor(r * len(pos) + 0.5))
                     order = sorted(pos, key=lambda p: (-sc[p], p))
@@ -179,7 +180,7 @@ def pin_sprint_invariants(lib):
             pos = [p for p in range(n) if (mod[i, p] != 0) == m]
             kin = [p for p in pos if p in ks]
             kout = [p for p in pos if p not in ks]
-            r = 0.7 if m == 0 else 0.8
+            r = float(np.float32(0.7 if m == 0 else 0.8))
             assert len(kin) == int(math.floor(r * len(pos) + 0.5))
             for a in kin:
                 for z in kout:
