@@ -31,7 +31,8 @@ BD_ERR_DEVICE_TIMEOUT = 4
 EXPORTED = ("bd_attn_fwd", "bd_attn_decode", "bd_attn_decode_workspace_bytes",
             "bd_attn_get_device_status", "bd_attn_status_string",
             "bd_spec_accept", "bd_cache_append", "bd_cache_crop",
-            "bd_sprint_prune", "bd_sprint_workspace_bytes")
+            "bd_sprint_prune", "bd_sprint_workspace_bytes", "bd_attn_bwd",
+            "bd_attn_bwd_workspace_bytes")
 
 
 class BdAttnError(RuntimeError):
@@ -66,6 +67,11 @@ def load(path: str = LIB_PATH):
     lib.bd_attn_get_device_status.argtypes = [vp]
     lib.bd_attn_status_string.restype = ctypes.c_char_p
     lib.bd_attn_status_string.argtypes = [i]
+    lib.bd_attn_bwd.restype = i
+    lib.bd_attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, i, f, vp, vp,
+                                           ctypes.c_size_t]
+    lib.bd_attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.bd_attn_bwd_workspace_bytes.argtypes = [i, i, i]
     lib.bd_spec_accept.restype = i
     lib.bd_spec_accept.argtypes = [vp, vp, vp, i, i, vp]
     lib.bd_cache_append.restype = i
@@ -109,6 +115,17 @@ def bd_attn_get_device_status(stream):
 
 def bd_attn_status_string(status):
     return load().bd_attn_status_string(status).decode()
+
+
+def bd_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, L, b, d,
+                scale, stream, workspace, workspace_bytes):
+    return load().bd_attn_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv,
+                              L, b, d, scale, stream, workspace,
+                              workspace_bytes)
+
+
+def bd_attn_bwd_workspace_bytes(B, Hq, L):
+    return int(load().bd_attn_bwd_workspace_bytes(B, Hq, L))
 
 
 def bd_spec_accept(draft, target, n_accept, B, b, stream):
@@ -191,6 +208,38 @@ def fwd(q, k, v, L: int, b: int, scale: float | None = None, out=None,
     if st != BD_OK:
         raise BdAttnError(st, "bd_attn_fwd")
     return out, lse
+
+
+def bwd(q, k, v, out, lse, dout, L: int, b: int, scale: float | None = None,
+        dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward of ``fwd``: gradients of q, k, v given dout (the gradient of
+    out), out and lse from the forward.  Returns (dq, dk, dv)."""
+    import torch
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if N != 2 * L or tuple(k.shape) != (B, Hkv, N, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if out.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, Hq, N):
+        raise ValueError("shape mismatch")
+    for t_, w in ((q, "q"), (k, "k"), (v, "v"), (out, "out"), (dout, "dout")):
+        _check(t_, torch.bfloat16, w)
+    _check(lse, torch.float32, "lse")
+    if scale is None:
+        scale = d ** -0.5
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nb = bd_attn_bwd_workspace_bytes(B, Hq, L)
+    if workspace is None:
+        workspace = torch.empty(nb, dtype=torch.uint8, device=q.device)
+    st = bd_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                     lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                     dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, L, b, d,
+                     float(scale), _stream_handle(stream), workspace.data_ptr(),
+                     workspace.numel() * workspace.element_size())
+    if st != BD_OK:
+        raise BdAttnError(st, "bd_attn_bwd")
+    return dq, dk, dv
 
 
 def decode(q_blk, k_cache, v_cache, cache_len, mode: int, out=None, lse=None,

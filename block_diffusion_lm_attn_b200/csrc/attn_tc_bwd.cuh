@@ -1,0 +1,913 @@
+// Backward of block-diffusion attention, training/prefill form, head dim
+// 128, on tcgen05 tensor cores (sm_100a).
+//
+// Training a block-diffusion LM minimises the BDLM loss ("LLaDA2.0-Uni",
+// section "Training objective and loss function", eq. L_BDLM); its gradient
+// flows through the attention over [x_t ; x_0] with the three-part block
+// mask ("Nemotron-Labs-Diffusion-8B-Base 3x decoding speed-up", section 1).
+// Given the forward's out and lse and the upstream gradient dO, for every
+// visible (query i, key j) pair of one head:
+//     P_ij  = exp(scale q_i.k_j - lse_i)
+//     dP_ij = dO_i . v_j,   D_i = dO_i . out_i,   dS_ij = P_ij (dP_ij - D_i)
+//     dV_j  = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,
+//     dQ_i  = scale sum_j dS_ij k_j
+// (q-heads of one GQA group add into their kv-head's dK and dV).
+//
+// Three kernels, no atomics:
+//   bd_bwd_prep_kernel   D_i and lse_i * log2(e) per query row (HBM-bound);
+//   bd_bwd_dkdv_kernel   one persistent CTA per SM; a work item is one
+//                        128-key tile of one kv-head; it walks the q-heads of
+//                        the group and, in 64-row steps, the query rows that
+//                        see the tile (the transpose of the forward's key
+//                        ranges), accumulating dV and dK in tensor memory;
+//   bd_bwd_dq_kernel     one persistent CTA per SM; a work item is one
+//                        128-row query tile, walking the forward's key
+//                        ranges, accumulating dQ in tensor memory.
+// The dQ pass recomputes S and dP (two of the five products) so that no
+// partial dQ ever leaves the SM.
+#pragma once
+
+#include "attn_tc_persist.cuh"
+
+namespace bd {
+
+struct BParams {
+    const bf16 *out, *dout;
+    const float *lse;
+    float *D;     // [B*Hq*2L] workspace: dO . out
+    float *lse2;  // [B*Hq*2L] workspace: lse * log2(e) (+inf for an empty row)
+    bf16 *dq, *dk, *dv;
+    int B, Hq, Hkv, L, b;
+    int qtiles;     // 128-row tiles per half
+    int sched_slot; // counter pair of this launch
+    float scale, scale_log2;
+};
+
+// ---------------------------------------------------------------------------
+// D and lse * log2(e), one warp per query row of 128 values.
+
+__global__ void __launch_bounds__(256)
+    bd_bwd_prep_kernel(const BParams p, long long rows)
+{
+    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows)
+        return;
+    const uint2 o = reinterpret_cast<const uint2 *>(p.out + r * kTcD)[lane];
+    const uint2 g = reinterpret_cast<const uint2 *>(p.dout + r * kTcD)[lane];
+    const uint32_t ow[2] = {o.x, o.y}, gw[2] = {g.x, g.y};
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        acc = fmaf(__uint_as_float(ow[t] << 16), __uint_as_float(gw[t] << 16), acc);
+        acc = fmaf(__uint_as_float(ow[t] & 0xffff0000u), __uint_as_float(gw[t] & 0xffff0000u), acc);
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1)
+        acc += __shfl_xor_sync(0xffffffffu, acc, s);
+    if (lane == 0) {
+        p.D[r] = acc;
+        const float l = p.lse[r];
+        p.lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Query rows that see key position c (the transpose of fwd_span):
+//   noisy key of block k : noisy rows [k b, k b + b)
+//   clean key of block k : noisy rows [(k+1) b, L)  U  clean rows [L + k b, 2L)
+__device__ __forceinline__ Span key_span(int L, int b, int c)
+{
+    Span s;
+    if (c < L) {
+        const int kb = c / b;
+        s.a0 = kb * b; s.a1 = kb * b + b; s.a2 = 0; s.a3 = 0;
+    } else {
+        const int kb = (c - L) / b;
+        s.a0 = (kb + 1) * b; s.a1 = L; s.a2 = L + kb * b; s.a3 = 2 * L;
+    }
+    return s;
+}
+
+constexpr int kBwdSub = 64; // query rows per step of the dK/dV kernel
+
+// Work item of the dK/dV kernel: (batch, kv-head) = w / R, rank r = w % R:
+// clean key tiles first (they are seen by the most query rows), idx
+// ascending, then noisy key tiles.
+struct KvItem {
+    int kvhead;       // batch * Hkv + kv-head
+    int qhead0;       // batch * Hq + first q-head of the group
+    int krow0, nkeys; // first key row (of 2L), valid keys (<= 128)
+    int lo0, hi0, lo1, hi1;     // query ranges
+    int flo0, fhi0, flo1, fhi1; // queries every key of the tile sees
+    int n0, n1;       // 64-row steps of range 0 / range 1 per q-head
+    int nt;           // steps of the item (all q-heads)
+};
+
+__device__ __forceinline__ long long kv_items(const BParams &p)
+{
+    return (long long)p.B * p.Hkv * 2 * p.qtiles;
+}
+
+__device__ __forceinline__ void kv_item(const BParams &p, int w, KvItem &it)
+{
+    const int R = 2 * p.qtiles;
+    const int bg = w / R, r = w % R;
+    const int clean = r < p.qtiles;
+    const int idx = clean ? r : r - p.qtiles;
+    const int bi = bg / p.Hkv, g = bg % p.Hkv;
+    const int G = p.Hq / p.Hkv;
+    it.kvhead = bg;
+    it.qhead0 = bi * p.Hq + g * G;
+    it.krow0 = (clean ? p.L : 0) + idx * kTcN;
+    it.nkeys = min(kTcN, p.L - idx * kTcN);
+    const Span first = key_span(p.L, p.b, it.krow0);
+    const Span last = key_span(p.L, p.b, it.krow0 + it.nkeys - 1);
+    it.lo0 = first.a0; it.hi0 = last.a1;
+    it.lo1 = first.a2; it.hi1 = last.a3;
+    it.flo0 = last.a0; it.fhi0 = first.a1;
+    it.flo1 = last.a2; it.fhi1 = first.a3;
+    it.n0 = it.hi0 > it.lo0 ? (it.hi0 - it.lo0 + kBwdSub - 1) / kBwdSub : 0;
+    it.n1 = it.hi1 > it.lo1 ? (it.hi1 - it.lo1 + kBwdSub - 1) / kBwdSub : 0;
+    it.nt = G * (it.n0 + it.n1);
+}
+
+// Step s of an item: q-head s / (n0 + n1), then range 0 or 1.
+__device__ __forceinline__ void kv_step(const KvItem &it, int s, int &qhead,
+                                        int &qs, int &rg)
+{
+    const int per = it.n0 + it.n1;
+    const int x = s / per, t = s % per;
+    qhead = it.qhead0 + x;
+    rg = t < it.n0 ? 0 : 1;
+    qs = rg == 0 ? it.lo0 + t * kBwdSub : it.lo1 + (t - it.n0) * kBwdSub;
+}
+
+// shared memory of the dK/dV kernel
+constexpr int kKvStages = 3;
+constexpr int kSubBytes = kBwdSub * kTcD * 2;              // 16 KB
+constexpr int kKvSmemK = 0;                                // K tile
+constexpr int kKvSmemV = kKvSmemK + kTileBytes;            // V tile
+constexpr int kKvSmemRing = kKvSmemV + kTileBytes;         // stages: Q, dO
+constexpr int kKvStageBytes = 2 * kSubBytes;
+constexpr int kKvSmemRows = kKvSmemRing + kKvStages * kKvStageBytes; // lse2, D
+constexpr int kKvRowsBytes = 2 * kBwdSub * 4;
+constexpr int kKvSmemBar = kKvSmemRows + kKvStages * kKvRowsBytes;
+constexpr int kKvSmemBytes = kKvSmemBar + 512 + 1024;
+static_assert(kKvStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
+static_assert(kKvSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
+
+constexpr int kBwdThreads = 192; // 4 compute warps, producer, MMA issuer
+
+// Roles: warps 0-3 compute P^T and dS^T (thread t = key row t = TMEM lane
+// t) and write dK, dV out; warp 4 loads (TMA for tiles, plain loads for the
+// per-row lse2 and D) and fetches work items; warp 5 issues the MMAs.
+// TMEM: dV [0,128), dK [128,256); two buffers x of S^T [256 + 128x, +64)
+// and dP^T [320 + 128x, +64); P^T (bf16) overwrites its S^T, dS^T its dP^T.
+// Per step s (64 query rows, buffer x = s & 1):
+//   S^T = K Q^T, dP^T = V dO^T into buffer x, then for step s - 1:
+//   dV += P^T dO, dK += dS^T Q from buffer x ^ 1 (tcgen05.mma from one
+//   thread execute in issue order, so buffer x is rewritten only after the
+//   products of step s - 2 that read it).
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bd_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_q64,
+                       const __grid_constant__ CUtensorMap tm_do64,
+                       const BParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + (base - raw_addr);
+
+    const uint32_t bar0 = base + kKvSmemBar;
+    const uint32_t bar_kvfull = bar0;        // K and V of the item landed
+    const uint32_t bar_kvfree = bar0 + 8;    // every product of the item read K, V
+    auto bar_full = [&](int s) { return bar0 + 16 + 8 * s; };  // stage landed
+    auto bar_empty = [&](int s) { return bar0 + 40 + 8 * s; }; // stage read
+    auto bar_sfull = [&](int x) { return bar0 + 64 + 8 * x; }; // S^T, dP^T ready
+    auto bar_pfull = [&](int x) { return bar0 + 80 + 8 * x; }; // P^T, dS^T written
+    const uint32_t bar_odone = bar0 + 96;  // the item's last dV, dK retired
+    const uint32_t bar_ofree = bar0 + 104; // dV, dK read out
+    const uint32_t bar_final = bar0 + 112;
+    const uint32_t bar_ifull0 = bar0 + 120;  // 4: work item published
+    const uint32_t bar_iempty0 = bar0 + 152; // 4: work item read by all roles
+    volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 256);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 384);
+    volatile uint32_t *tmem_slot =
+        reinterpret_cast<volatile uint32_t *>(sbase + kKvSmemBar + 392);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kvfull, 1);
+        mbar_init(bar_kvfree, 1);
+        for (int s = 0; s < kKvStages; ++s) {
+            mbar_init(bar_full(s), 2); // expect_tx arrival + lse2/D arrival
+            mbar_init(bar_empty(s), 1);
+        }
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(bar_sfull(x), 1);
+            mbar_init(bar_pfull(x), 128);
+        }
+        mbar_init(bar_odone, 1);
+        mbar_init(bar_ofree, 128);
+        mbar_init(bar_final, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_ifull0 + 8 * i, 1);
+            mbar_init(bar_iempty0 + 8 * i, 129); // MMA + 128 compute threads
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32((const void *)tmem_slot)), "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_dv = tmem, t_dk = tmem + 128;
+    auto t_st = [&](int x) { return tmem + 256 + 128 * (uint32_t)x; };
+    auto t_dp = [&](int x) { return tmem + 320 + 128 * (uint32_t)x; };
+
+    KvItem it;
+    auto next_item = [&](int si, bool producer, bool &ok) -> bool {
+        const int slot = si & 3;
+        int w;
+        if (producer) {
+            if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
+                                             (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
+                return false;
+            const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
+            w = (long long)t < kv_items(p) ? (int)t : -1;
+            item_ring[slot] = w;
+            mbar_arrive(bar_ifull0 + 8 * slot);
+        } else {
+            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+                return false;
+            w = item_ring[slot];
+            mbar_arrive(bar_iempty0 + 8 * slot);
+        }
+        if (w < 0)
+            return false;
+        kv_item(p, w, it);
+        return true;
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------------ producer
+        bool ok = true;
+        int si = 0;
+        long long g = 0, iss = 0; // running step counter, steps issued
+        const long long nrows_all = (long long)p.B * p.Hq * 2 * p.L;
+        for (;;) {
+            bool got = false;
+            if (lane == 0)
+                got = next_item(si, true, ok);
+            __syncwarp();
+            got = __shfl_sync(0xffffffffu, got, 0);
+            if (!got)
+                break;
+            if (lane != 0)
+                kv_item(p, item_ring[si & 3], it);
+            if (lane == 0) {
+                // K, V of item si - 1 are no longer read
+                if (si >= 1 && !(ok = mbar_wait(bar_kvfree, (uint32_t)((si - 1) & 1), abort_flag)))
+                    got = false;
+                if (ok) {
+                    mbar_expect_tx(bar_kvfull, 2 * kTileBytes);
+                    tma_load_3d(base + kKvSmemK, &tm_k, 0, it.krow0, it.kvhead, bar_kvfull);
+                    tma_load_3d(base + kKvSmemK + kHalfTileBytes, &tm_k, 64, it.krow0, it.kvhead,
+                                bar_kvfull);
+                    tma_load_3d(base + kKvSmemV, &tm_v, 0, it.krow0, it.kvhead, bar_kvfull);
+                    tma_load_3d(base + kKvSmemV + kHalfTileBytes, &tm_v, 64, it.krow0, it.kvhead,
+                                bar_kvfull);
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok)
+                break;
+            ++si;
+            for (int s = 0; s < it.nt && ok; ++s, ++g) {
+                const int st = (int)(g % kKvStages);
+                int qhead, qs, rg;
+                kv_step(it, s, qhead, qs, rg);
+                if (lane == 0 && g >= kKvStages)
+                    ok = mbar_wait(bar_empty(st), (uint32_t)(((g - kKvStages) / kKvStages) & 1),
+                                   abort_flag);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok)
+                    break;
+                const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
+                if (lane == 0) {
+                    mbar_expect_tx(bar_full(st), 2 * kSubBytes);
+                    tma_load_3d(sb, &tm_q64, 0, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes / 2, &tm_q64, 64, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes, &tm_do64, 0, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes + kSubBytes / 2, &tm_do64, 64, qs, qhead,
+                                bar_full(st));
+                    iss = g + 1;
+                }
+                // lse2 and D of the 64 rows; rows outside the range get
+                // lse2 = +inf (P = 0)
+                const int hi = rg == 0 ? it.hi0 : it.hi1;
+                float *sl = reinterpret_cast<float *>(sbase + kKvSmemRows + st * kKvRowsBytes);
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int c = lane + 32 * u;
+                    const long long row = (long long)qhead * 2 * p.L + qs + c;
+                    const bool v = qs + c < hi && row < nrows_all;
+                    sl[c] = v ? p.lse2[row] : INFINITY;
+                    sl[kBwdSub + c] = v ? p.D[row] : 0.f;
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_full(st));
+            }
+        }
+        if (lane == 0) {
+            __threadfence();
+            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
+                g_sched_next[p.sched_slot] = 0;
+                g_sched_done[p.sched_slot] = 0;
+                __threadfence();
+            }
+            const long long c0 = clock64();
+            auto drain = [&](uint32_t bar, uint32_t par) {
+                while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}
+            };
+            if (si >= 1)
+                drain(bar_kvfull, (uint32_t)((si - 1) & 1));
+            for (long long x = iss > kKvStages ? iss - kKvStages : 0; x < iss; ++x)
+                drain(bar_full((int)(x % kKvStages)), (uint32_t)((x / kKvStages) & 1));
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(kTcM, kBwdSub, 0);  // S^T, dP^T
+            constexpr uint32_t idesc_g = idesc_bf16(kTcM, kTcD, 1);     // dV, dK
+            bool ok = true;
+            int si = 0;
+            long long g = 0;
+            auto issue_sdp = [&](long long gg) {
+                const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
+                const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
+                    tc_mma_ss(t_st(x), smem_desc_sw128(base + kKvSmemK + ao, 16, 1024),
+                              smem_desc_sw128(sb + bo, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
+                    tc_mma_ss(t_dp(x), smem_desc_sw128(base + kKvSmemV + ao, 16, 1024),
+                              smem_desc_sw128(sb + kSubBytes + bo, 16, 1024), idesc_s,
+                              kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar_sfull(x));
+            };
+            auto issue_grad = [&](long long gg, bool first) {
+                const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
+                const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBwdSub / 16; ++kk) {
+                    const uint64_t bdo = smem_desc_sw128(sb + kSubBytes + kk * 2048, kSubBytes / 2, 1024);
+                    tc_mma_ts(t_dv, t_st(x) + kk * 8, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kBwdSub / 16; ++kk) {
+                    const uint64_t bq = smem_desc_sw128(sb + kk * 2048, kSubBytes / 2, 1024);
+                    tc_mma_ts(t_dk, t_dp(x) + kk * 8, bq, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_empty(st));
+            };
+            while (ok && next_item(si, false, ok)) {
+                if (!(ok = mbar_wait(bar_kvfull, (uint32_t)(si & 1), abort_flag)))
+                    break;
+                tc_fence_after();
+                for (int s = 0; s <= it.nt && ok; ++s) {
+                    if (s < it.nt) {
+                        const long long gg = g + s;
+                        if (!(ok = mbar_wait(bar_full((int)(gg % kKvStages)),
+                                             (uint32_t)((gg / kKvStages) & 1), abort_flag)))
+                            break;
+                        tc_fence_after();
+                        issue_sdp(gg);
+                    }
+                    if (s >= 1) {
+                        const long long gp = g + s - 1;
+                        if (s == 1 && si >= 1 &&
+                            !(ok = mbar_wait(bar_ofree, (uint32_t)((si - 1) & 1), abort_flag)))
+                            break;
+                        if (!(ok = mbar_wait(bar_pfull((int)(gp & 1)), (uint32_t)((gp >> 1) & 1),
+                                             abort_flag)))
+                            break;
+                        tc_fence_after();
+                        issue_grad(gp, s == 1);
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit(bar_kvfree);
+                tc_commit(bar_odone);
+                g += it.nt;
+                ++si;
+            }
+            tc_commit(bar_final);
+            const long long c0 = clock64();
+            while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
+        }
+    } else {
+        // ------------------------------------------ P^T, dS^T and epilogue
+        const int row = threadIdx.x; // key row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        long long g = 0;
+        int si = 0;
+        for (;;) {
+            const bool got = next_item(si, false, ok);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!got || !ok)
+                break;
+            const Span ksp = key_span(p.L, p.b, it.krow0 + min(row, it.nkeys - 1));
+            for (int s = 0; s < it.nt; ++s) {
+                const long long gg = g + s;
+                const int x = (int)(gg & 1), st = (int)(gg % kKvStages);
+                int qhead, qs, rg;
+                kv_step(it, s, qhead, qs, rg);
+                ok = __all_sync(0xffffffffu,
+                                mbar_wait(bar_sfull(x), (uint32_t)((gg >> 1) & 1), abort_flag));
+                if (!ok)
+                    break;
+                // the stage's lse2 / D (written by the producer before its
+                // arrival on the stage barrier, which the MMA thread waited
+                // for before issuing this step's products)
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_full(st),
+                                                       (uint32_t)((gg / kKvStages) & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                uint32_t sr[64], dr[64];
+                tmem_ld32(t_st(x) + lane_off, sr);
+                tmem_ld32(t_st(x) + lane_off + 32, sr + 32);
+                tmem_ld32(t_dp(x) + lane_off, dr);
+                tmem_ld32(t_dp(x) + lane_off + 32, dr + 32);
+                tmem_wait_ld();
+                const float *sl = reinterpret_cast<const float *>(
+                    sbase + kKvSmemRows + st * kKvRowsBytes);
+                const int hi = rg == 0 ? it.hi0 : it.hi1;
+                const int flo = rg == 0 ? it.flo0 : it.flo1;
+                const int fhi = rg == 0 ? it.fhi0 : it.fhi1;
+                const bool full = qs >= flo && qs + kBwdSub <= fhi && qs + kBwdSub <= hi;
+                uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
+                if (!full) {
+                    const int e = min(hi, qs + kBwdSub);
+                    const int lo0 = max(ksp.a0, qs) - qs, hi0 = min(ksp.a1, e) - qs;
+                    const int lo1 = max(ksp.a2, qs) - qs, hi1 = min(ksp.a3, e) - qs;
+#pragma unroll
+                    for (int w = 0; w < 2; ++w)
+                        mw[w] = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
+                }
+                uint32_t pk[32], dk[32];
+#pragma unroll
+                for (int c = 0; c < kBwdSub; c += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4 *>(sl + c);
+                    const float4 d4 = *reinterpret_cast<const float4 *>(sl + kBwdSub + c);
+                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pv[4], dv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int cc = c + u;
+                        float xx = fmaf(__uint_as_float(sr[cc]), sl2, -la[u]);
+                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u))
+                            xx = -INFINITY;
+                        pv[u] = ex2(xx);
+                        dv[u] = pv[u] * (__uint_as_float(dr[cc]) - da[u]);
+                    }
+                    pk[c / 2] = pack_bf16x2(pv[0], pv[1]);
+                    pk[c / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                    dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
+                    dk[c / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
+                }
+                tmem_st16(t_st(x) + lane_off, pk);
+                tmem_st16(t_st(x) + lane_off + 16, pk + 16);
+                tmem_st16(t_dp(x) + lane_off, dk);
+                tmem_st16(t_dp(x) + lane_off + 16, dk + 16);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_pfull(x));
+            }
+            if (!ok)
+                break;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_odone, (uint32_t)(si & 1), abort_flag));
+            if (!ok)
+                break;
+            tc_fence_after();
+            // epilogue: dV and scale * dK, bf16, one row per thread
+            const bool valid = row < it.nkeys;
+            const size_t grow = (size_t)it.kvhead * 2 * p.L + it.krow0 + row;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t tb = (which == 0 ? t_dv : t_dk) + lane_off;
+                const float mul = which == 0 ? 1.f : p.scale;
+                bf16 *dst = (which == 0 ? p.dv : p.dk) + grow * kTcD;
+#pragma unroll
+                for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                    uint32_t o[32];
+                    tmem_ld32(tb + q4 * 32, o);
+                    tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 v4;
+                            v4.x = pack_bf16x2(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul);
+                            v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * mul, __uint_as_float(o[i + 3]) * mul);
+                            v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * mul, __uint_as_float(o[i + 5]) * mul);
+                            v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * mul, __uint_as_float(o[i + 7]) * mul);
+                            reinterpret_cast<uint4 *>(dst)[q4 * 4 + i / 8] = v4;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_ofree);
+            g += it.nt;
+            ++si;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dQ: one 128-row query tile per work item, the forward's key ranges.
+
+constexpr int kDqSmemQ = 0;                          // Q tile
+constexpr int kDqSmemDO = kDqSmemQ + kTileBytes;     // dO tile
+constexpr int kDqSmemRing = kDqSmemDO + kTileBytes;  // 2 stages of K, V
+constexpr int kDqSmemBar = kDqSmemRing + 2 * 2 * kTileBytes;
+constexpr int kDqSmemBytes = kDqSmemBar + 512 + 1024;
+static_assert(kDqSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
+
+// Roles: warps 0-3 compute dS (thread t = query row t) and write dQ out;
+// warp 4 loads and fetches items; warp 5 issues the MMAs.  TMEM: S [0,128),
+// dP [128,256), dQ [256,384), two dS buffers (bf16) [384,448), [448,512).
+// Per key tile j: S = Q K^T and dP = dO V^T (after the compute warps have
+// read S, dP of tile j - 1 into registers), then dQ += dS(j - 1) K(j - 1).
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bd_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const BParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base = (raw_addr + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + (base - raw_addr);
+
+    const uint32_t bar0 = base + kDqSmemBar;
+    const uint32_t bar_qfull = bar0;      // Q and dO landed
+    const uint32_t bar_qfree = bar0 + 8;  // every S, dP of the item retired
+    auto bar_kvfull = [&](int s) { return bar0 + 16 + 8 * s; };
+    auto bar_kvempty = [&](int s) { return bar0 + 32 + 8 * s; };
+    const uint32_t bar_sfull = bar0 + 48;  // S, dP ready
+    const uint32_t bar_sfree = bar0 + 56;  // S, dP read into registers (128)
+    auto bar_dsfull = [&](int x) { return bar0 + 64 + 8 * x; };  // (128)
+    auto bar_dsfree = [&](int x) { return bar0 + 80 + 8 * x; };
+    const uint32_t bar_qdone = bar0 + 96;  // the item's last dQ retired
+    const uint32_t bar_dqfree = bar0 + 104; // dQ read out (128)
+    const uint32_t bar_final = bar0 + 112;
+    const uint32_t bar_ifull0 = bar0 + 120;
+    const uint32_t bar_iempty0 = bar0 + 152;
+    volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 256);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 384);
+    volatile uint32_t *tmem_slot =
+        reinterpret_cast<volatile uint32_t *>(sbase + kDqSmemBar + 392);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(bar_qfull, 1);
+        mbar_init(bar_qfree, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_kvfull(s), 1);
+            mbar_init(bar_kvempty(s), 1);
+            mbar_init(bar_dsfull(s), 128);
+            mbar_init(bar_dsfree(s), 1);
+        }
+        mbar_init(bar_sfull, 1);
+        mbar_init(bar_sfree, 128);
+        mbar_init(bar_qdone, 1);
+        mbar_init(bar_dqfree, 128);
+        mbar_init(bar_final, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar_ifull0 + 8 * i, 1);
+            mbar_init(bar_iempty0 + 8 * i, 129);
+        }
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32((const void *)tmem_slot)), "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+    auto t_ds = [&](int x) { return tmem + 384 + 64 * (uint32_t)x; };
+
+    // the forward's work list: (batch * Hq + head, query tile), heaviest first
+    PParams fp = {};
+    fp.B = p.B; fp.Hq = p.Hq; fp.Hkv = p.Hkv; fp.L = p.L; fp.b = p.b;
+    fp.qtiles = p.qtiles;
+    Seg sg;
+    auto next_item = [&](int si, bool producer, bool &ok) -> bool {
+        const int slot = si & 3;
+        int w;
+        if (producer) {
+            if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
+                                             (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
+                return false;
+            const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
+            w = (long long)t < FwdSource::items(fp) ? (int)t : -1;
+            item_ring[slot] = w;
+            mbar_arrive(bar_ifull0 + 8 * slot);
+        } else {
+            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+                return false;
+            w = item_ring[slot];
+            mbar_arrive(bar_iempty0 + 8 * slot);
+        }
+        if (w < 0)
+            return false;
+        FwdSource::item(fp, w, sg);
+        return true;
+    };
+    auto key_start = [&](int t) {
+        return t < sg.n0 ? sg.lo0 + t * kTcN : sg.lo1 + (t - sg.n0) * kTcN;
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            bool ok = true;
+            int si = 0;
+            long long g = 0, iss = 0;
+            while (ok && next_item(si, true, ok)) {
+                if (si >= 1 && !(ok = mbar_wait(bar_qfree, (uint32_t)((si - 1) & 1), abort_flag)))
+                    break;
+                mbar_expect_tx(bar_qfull, 2 * kTileBytes);
+                tma_load_3d(base + kDqSmemQ, &tm_q, 0, sg.qrow0, sg.qhead, bar_qfull);
+                tma_load_3d(base + kDqSmemQ + kHalfTileBytes, &tm_q, 64, sg.qrow0, sg.qhead, bar_qfull);
+                tma_load_3d(base + kDqSmemDO, &tm_do, 0, sg.qrow0, sg.qhead, bar_qfull);
+                tma_load_3d(base + kDqSmemDO + kHalfTileBytes, &tm_do, 64, sg.qrow0, sg.qhead,
+                            bar_qfull);
+                ++si;
+                for (int t = 0; t < sg.nt; ++t, ++g) {
+                    const int s = (int)(g & 1);
+                    if (g >= 2 && !(ok = mbar_wait(bar_kvempty(s), (uint32_t)(((g - 2) >> 1) & 1),
+                                                   abort_flag)))
+                        break;
+                    const int ks = key_start(t);
+                    const uint32_t kb = base + kDqSmemRing + (uint32_t)s * 2 * kTileBytes;
+                    mbar_expect_tx(bar_kvfull(s), 2 * kTileBytes);
+                    tma_load_3d(kb, &tm_k, 0, ks, sg.kvhead, bar_kvfull(s));
+                    tma_load_3d(kb + kHalfTileBytes, &tm_k, 64, ks, sg.kvhead, bar_kvfull(s));
+                    tma_load_3d(kb + kTileBytes, &tm_v, 0, ks, sg.kvhead, bar_kvfull(s));
+                    tma_load_3d(kb + kTileBytes + kHalfTileBytes, &tm_v, 64, ks, sg.kvhead,
+                                bar_kvfull(s));
+                    iss = g + 1;
+                }
+            }
+            __threadfence();
+            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
+                g_sched_next[p.sched_slot] = 0;
+                g_sched_done[p.sched_slot] = 0;
+                __threadfence();
+            }
+            const long long c0 = clock64();
+            auto drain = [&](uint32_t bar, uint32_t par) {
+                while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}
+            };
+            if (si >= 1)
+                drain(bar_qfull, (uint32_t)((si - 1) & 1));
+            for (long long x = iss > 2 ? iss - 2 : 0; x < iss; ++x)
+                drain(bar_kvfull((int)(x & 1)), (uint32_t)((x >> 1) & 1));
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(kTcM, kTcN, 0);
+            constexpr uint32_t idesc_q = idesc_bf16(kTcM, kTcD, 1);
+            bool ok = true;
+            int si = 0;
+            long long j = 0; // running key-tile counter
+            auto issue_sdp = [&](long long jg) {
+                const uint32_t kb = base + kDqSmemRing + (uint32_t)(jg & 1) * 2 * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    tc_mma_ss(t_s, smem_desc_sw128(base + kDqSmemQ + off, 16, 1024),
+                              smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    tc_mma_ss(t_dp, smem_desc_sw128(base + kDqSmemDO + off, 16, 1024),
+                              smem_desc_sw128(kb + kTileBytes + off, 16, 1024), idesc_s,
+                              kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar_sfull);
+            };
+            auto issue_dq = [&](long long jg, bool first) {
+                const uint32_t kb = base + kDqSmemRing + (uint32_t)(jg & 1) * 2 * kTileBytes;
+                const int x = (int)(jg & 1);
+#pragma unroll
+                for (int kk = 0; kk < kTcN / 16; ++kk) {
+                    const uint64_t bk = smem_desc_sw128(kb + kk * 2048, kHalfTileBytes, 1024);
+                    tc_mma_ts(t_dq, t_ds(x) + kk * 8, bk, idesc_q, (!first || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar_dsfree(x));
+                tc_commit(bar_kvempty(x));
+            };
+            while (ok && next_item(si, false, ok)) {
+                if (!(ok = mbar_wait(bar_qfull, (uint32_t)(si & 1), abort_flag)))
+                    break;
+                for (int t = 0; t <= sg.nt && ok; ++t) {
+                    const long long jg = j + t;
+                    if (t < sg.nt) {
+                        if (!(ok = mbar_wait(bar_kvfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
+                                             abort_flag)))
+                            break;
+                        // S, dP of the previous tile are in registers
+                        if (jg >= 1 && !(ok = mbar_wait(bar_sfree, (uint32_t)((jg - 1) & 1),
+                                                        abort_flag)))
+                            break;
+                        tc_fence_after();
+                        issue_sdp(jg);
+                        if (t == sg.nt - 1)
+                            tc_commit(bar_qfree);
+                    }
+                    if (t >= 1) {
+                        const long long jp = jg - 1;
+                        if (t == 1 && si >= 1 &&
+                            !(ok = mbar_wait(bar_dqfree, (uint32_t)((si - 1) & 1), abort_flag)))
+                            break;
+                        if (!(ok = mbar_wait(bar_dsfull((int)(jp & 1)), (uint32_t)((jp >> 1) & 1),
+                                             abort_flag)))
+                            break;
+                        tc_fence_after();
+                        issue_dq(jp, t == 1);
+                    }
+                }
+                if (!ok)
+                    break;
+                tc_commit(bar_qdone);
+                j += sg.nt;
+                ++si;
+            }
+            tc_commit(bar_final);
+            const long long c0 = clock64();
+            while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
+        }
+    } else {
+        // ---------------------------------------------- dS and epilogue
+        const int row = threadIdx.x;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        long long j = 0;
+        int si = 0;
+        for (;;) {
+            const bool got = next_item(si, false, ok);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!got || !ok)
+                break;
+            const int rl = min(row, sg.nrows - 1);
+            const Span sp = fwd_span(p.L, p.b, sg.qrow0 + rl);
+            const size_t grow = (size_t)sg.qhead * 2 * p.L + sg.qrow0 + row;
+            const bool valid = row < sg.nrows;
+            const float lse2 = valid ? p.lse2[grow] : INFINITY;
+            const float Dr = valid ? p.D[grow] : 0.f;
+            for (int t = 0; t < sg.nt; ++t) {
+                const long long jg = j + t;
+                const int x = (int)(jg & 1);
+                const bool r0 = t < sg.n0;
+                const int ks = key_start(t);
+                const int khi = r0 ? sg.hi0 : sg.hi1;
+                const int flo = r0 ? sg.flo0 : sg.flo1;
+                const int fhi = r0 ? sg.fhi0 : sg.fhi1;
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_sfull, (uint32_t)(jg & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
+                uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+                if (!full) {
+                    const int e = min(khi, ks + kTcN);
+                    const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
+                    const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        mw[w] = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
+                }
+                // dS buffer x was last read by dQ of tile jg - 2 (issued
+                // while this warp worked on tile jg - 1)
+                if (jg >= 2) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(bar_dsfree(x), (uint32_t)(((jg - 2) >> 1) & 1),
+                                                           abort_flag));
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t sr[64], dr[64], pk[32];
+                    tmem_ld32(t_s + lane_off + 64 * h, sr);
+                    tmem_ld32(t_s + lane_off + 64 * h + 32, sr + 32);
+                    tmem_ld32(t_dp + lane_off + 64 * h, dr);
+                    tmem_ld32(t_dp + lane_off + 64 * h + 32, dr + 32);
+                    tmem_wait_ld();
+                    if (h == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar_sfree); // S, dP may be overwritten
+                    }
+#pragma unroll
+                    for (int c = 0; c < 64; c += 2) {
+                        const int cc = 64 * h + c;
+                        float x0 = fmaf(__uint_as_float(sr[c]), sl2, -lse2);
+                        float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2);
+                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u))
+                            x0 = -INFINITY;
+                        if (!((mw[(cc + 1) >> 5] >> ((cc + 1) & 31)) & 1u))
+                            x1 = -INFINITY;
+                        const float p0 = ex2(x0), p1 = ex2(x1);
+                        pk[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[c]) - Dr),
+                                                p1 * (__uint_as_float(dr[c + 1]) - Dr));
+                    }
+                    tmem_st16(t_ds(x) + lane_off + 32 * h, pk);
+                    tmem_st16(t_ds(x) + lane_off + 32 * h + 16, pk + 16);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(bar_dsfull(x));
+            }
+            if (!ok)
+                break;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_qdone, (uint32_t)(si & 1), abort_flag));
+            if (!ok)
+                break;
+            tc_fence_after();
+#pragma unroll
+            for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                uint32_t o[32];
+                tmem_ld32(t_dq + lane_off + q4 * 32, o);
+                tmem_wait_ld();
+                if (valid) {
+                    const float mul = p.scale;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul);
+                        v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * mul, __uint_as_float(o[i + 3]) * mul);
+                        v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * mul, __uint_as_float(o[i + 5]) * mul);
+                        v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * mul, __uint_as_float(o[i + 7]) * mul);
+                        reinterpret_cast<uint4 *>(p.dq + grow * kTcD)[q4 * 4 + i / 8] = v4;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar_dqfree);
+            j += sg.nt;
+            ++si;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+} // namespace bd

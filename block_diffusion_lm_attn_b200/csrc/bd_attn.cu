@@ -21,6 +21,7 @@
 #include "attn_tc.cuh"
 #include "attn_tc_persist.cuh"
 #include "attn_tc_pair.cuh"
+#include "attn_tc_bwd.cuh"
 #include "bd_common.cuh"
 #include "cache_ops.cuh"
 
@@ -192,16 +193,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // 3-D map over a row-major bf16 tensor [n2][n1][128]: boxes of 64 columns x
-// 128 rows x 1, 128-byte swizzle, rows beyond n1 read as zero.
-bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
-                      uint64_t n2)
+// box_rows rows x 1, 128-byte swizzle, rows beyond n1 read as zero.
+bool make_map_rows(CUtensorMap *m, const void *base, uint64_t n1, uint64_t n2,
+                   uint32_t box_rows)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
     cuuint64_t dims[3] = {128, n1, n2};
     cuuint64_t strides[2] = {128 * 2, 128 * 2 * n1};
-    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                      const_cast<void *>(base), dims, strides, box, estr,
@@ -209,6 +210,20 @@ bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
+                      uint64_t n2)
+{
+    return make_map_rows(m, base, n1, n2, 128);
+}
+
+// Counter pair of the next persistent launch that hands out work items
+// dynamically (forward, and both backward passes).
+std::atomic<unsigned int> g_launches{0};
+int next_sched_slot()
+{
+    return (int)(g_launches.fetch_add(1u) % bd::kSchedSlots);
 }
 
 template <int KIND>
@@ -406,8 +421,7 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
             !make_map_rows128(&mk, k, N, (uint64_t)B * Hkv) ||
             !make_map_rows128(&mv, v, N, (uint64_t)B * Hkv))
             return BD_ERR_CUDA;
-        static std::atomic<unsigned int> launches{0};
-        p.sched_slot = (int)(launches.fetch_add(1u) % bd::kSchedSlots);
+        p.sched_slot = next_sched_slot();
         // two query heads of one GQA group per CTA when the group size is even
         const bool pair = (Hq / Hkv) % 2 == 0 && pair_kernel_usable();
         const long long items = (long long)B * (pair ? Hq / 2 : Hq) * 2 * p.qtiles;
@@ -438,6 +452,92 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
     case 32: return launch_fwd_mma<32>(p, stream);
     default: return launch_fwd_mma<64>(p, stream);
     }
+}
+
+size_t bd_attn_bwd_workspace_bytes(int B, int Hq, int L)
+{
+    if (B <= 0 || Hq <= 0 || L <= 0)
+        return 0;
+    return 2 * round256((size_t)B * Hq * 2 * L * sizeof(float));
+}
+
+bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
+                      const void *out, const float *lse, const void *dout,
+                      void *dq, void *dk, void *dv, int B, int Hq, int Hkv,
+                      int L, int b, int d, float scale, cudaStream_t stream,
+                      void *workspace, size_t workspace_bytes)
+{
+    if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return BD_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(lse) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+        !aligned16(dv) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return BD_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || b <= 0 || d <= 0)
+        return BD_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || L % b != 0)
+        return BD_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || !std::isfinite(scale))
+        return BD_ERR_INVALID_ARG;
+    if (workspace_bytes < bd_attn_bwd_workspace_bytes(B, Hq, L))
+        return BD_ERR_INVALID_ARG;
+    if (d != 128)
+        return BD_ERR_UNSUPPORTED;
+    if ((long long)B * Hq > 65535LL || 2LL * L * (long long)B * Hq * d > (1LL << 40))
+        return BD_ERR_UNSUPPORTED;
+
+    bd::BParams p = {};
+    p.out = static_cast<const bf16 *>(out);
+    p.dout = static_cast<const bf16 *>(dout);
+    p.lse = lse;
+    const size_t rows = (size_t)B * Hq * 2 * L;
+    p.D = static_cast<float *>(workspace);
+    p.lse2 = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                       round256(rows * sizeof(float)));
+    p.dq = static_cast<bf16 *>(dq);
+    p.dk = static_cast<bf16 *>(dk);
+    p.dv = static_cast<bf16 *>(dv);
+    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
+    p.qtiles = (int)cdiv(L, bd::kTcM);
+    p.scale = scale;
+    p.scale_log2 = scale * bd::kLog2e;
+
+    CUtensorMap mq, mq64, mdo, mdo64, mk, mv;
+    const uint64_t N = 2ull * L;
+    if (!make_map_rows(&mq, q, N, (uint64_t)B * Hq, 128) ||
+        !make_map_rows(&mq64, q, N, (uint64_t)B * Hq, bd::kBwdSub) ||
+        !make_map_rows(&mdo, dout, N, (uint64_t)B * Hq, 128) ||
+        !make_map_rows(&mdo64, dout, N, (uint64_t)B * Hq, bd::kBwdSub) ||
+        !make_map_rows(&mk, k, N, (uint64_t)B * Hkv, 128) ||
+        !make_map_rows(&mv, v, N, (uint64_t)B * Hkv, 128))
+        return BD_ERR_CUDA;
+
+    bd::bd_bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, (long long)rows);
+    if (cudaGetLastError() != cudaSuccess)
+        return BD_ERR_CUDA;
+
+    const int G0 = persistent_grid();
+    {
+        p.sched_slot = next_sched_slot();
+        const long long items = (long long)B * Hkv * 2 * p.qtiles;
+        const int G = items < G0 ? (int)items : G0;
+        if (set_smem<bd::bd_bwd_dkdv_kernel>(bd::kKvSmemBytes) != BD_OK)
+            return BD_ERR_CUDA;
+        bd::bd_bwd_dkdv_kernel<<<G, bd::kBwdThreads, bd::kKvSmemBytes, stream>>>(mk, mv, mq64,
+                                                                               mdo64, p);
+        if (cudaGetLastError() != cudaSuccess)
+            return BD_ERR_CUDA;
+    }
+    {
+        p.sched_slot = next_sched_slot();
+        const long long items = (long long)B * Hq * 2 * p.qtiles;
+        const int G = items < G0 ? (int)items : G0;
+        if (set_smem<bd::bd_bwd_dq_kernel>(bd::kDqSmemBytes) != BD_OK)
+            return BD_ERR_CUDA;
+        bd::bd_bwd_dq_kernel<<<G, bd::kBwdThreads, bd::kDqSmemBytes, stream>>>(mq, mdo, mk, mv,
+                                                                             p);
+    }
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
 }
 
 size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int d,

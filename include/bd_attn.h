@@ -90,6 +90,46 @@ BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *
                       float scale, struct CUstream_st *stream);
 
 /*
+ * Backward of the training / prefill block-diffusion attention.
+ *
+ * Defines: the gradient that the BDLM training objective of "LLaDA2.0-Uni"
+ * (discuss.pytorch.kr), section "Training objective and loss function", eq.
+ * L_BDLM, sends through the attention of bd_attn_fwd (same mask, same
+ * layouts).  For every visible (query i, key j) pair of one head, with
+ * P_ij = exp(scale q_i.k_j - lse_i) and D_i = dout_i . out_i:
+ *     dv_j = sum_i P_ij dout_i,
+ *     dS_ij = P_ij (dout_i . v_j - D_i),
+ *     dq_i = scale sum_j dS_ij k_j,   dk_j = scale sum_i dS_ij q_i;
+ * the q-heads of a GQA group add into their kv-head's dk and dv.  The lse
+ * side output of the forward is treated as a constant (no gradient into it).
+ *
+ *   q, out, dout [B, Hq,  2L, d] bf16   (read; out and lse as written by
+ *   lse          [B, Hq,  2L]    fp32    bd_attn_fwd for these q, k, v)
+ *   k, v         [B, Hkv, 2L, d] bf16   (read)
+ *   dq           [B, Hq,  2L, d] bf16   (written)
+ *   dk, dv       [B, Hkv, 2L, d] bf16   (written)
+ *   workspace    DEVICE scratch of bd_attn_bwd_workspace_bytes(B, Hq, L)
+ *                bytes, 256-byte aligned (per-row D and lse * log2 e)
+ *
+ * Three kernels on `stream`: a per-row pass, a dK/dV pass over key tiles and
+ * a dQ pass over query tiles; nothing is allocated and no atomics are used,
+ * so results are deterministic.  Concurrency as for bd_attn_fwd (each pass
+ * takes one of the 64 scheduling counter pairs).
+ *
+ * Errors: as bd_attn_fwd, plus BD_ERR_INVALID_ARG for a null or misaligned
+ * workspace or one smaller than required; BD_ERR_UNSUPPORTED for d != 128.
+ */
+BD_API bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
+                             const void *out, const float *lse,
+                             const void *dout, void *dq, void *dk, void *dv,
+                             int B, int Hq, int Hkv, int L, int b, int d,
+                             float scale, struct CUstream_st *stream,
+                             void *workspace, size_t workspace_bytes);
+
+/* Bytes of scratch bd_attn_bwd needs (0 on bad sizes).  Host only. */
+BD_API size_t bd_attn_bwd_workspace_bytes(int B, int Hq, int L);
+
+/*
  * Block-decode block-diffusion attention.
  *
  * Defines: a block of b noisy queries attends to the cached clean prefix and

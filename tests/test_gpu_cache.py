@@ -112,7 +112,7 @@ def check_sprint(k, v, conf, mod, cl, alpha, kt, ki):
         # none, so the integers must match exactly
         for m in (0, 1):
             s_m = np.sort(rs[i, :n][(mod[i, :n].numpy() != 0) == m])[::-1]
-            r = kt if m == 0 else ki
+            r = float(np.float32(kt if m == 0 else ki))  # the interface takes fp32
             want = int(math.floor(r * len(s_m) + 0.5))
             if 0 < want < len(s_m):
                 assert s_m[want - 1] - s_m[want] > 1e-9, "near-tie in the inputs"

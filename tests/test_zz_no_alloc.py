@@ -1,13 +1,20 @@
 """Block decode through bd_attn_decode_noalloc, the entry point for callers
 that cannot allocate device memory at decode time (its split-KV scratch is a
 fixed array inside the library).  Two calls in a row, with different inputs,
-each compared with bd_attn_decode on the same inputs.  Collected last so that
-a run stopping at the first failure has already run every other test."""
+each compared with bd_attn_decode on the same inputs, and once directly with
+the fp64 oracle; both head-dim paths (the d = 128 stream-K layout and the
+d = 64 split-KV layout share the array); and a call inside a captured CUDA
+graph in global capture mode, where any allocation would fail the capture.
+Collected last so that a run stopping at the first failure has already run
+every other test."""
+import math
+
 import numpy as np
 import pytest
 import torch
 
 import bd_inputs
+import oracle
 import block_diffusion_lm_attn_b200 as bd
 from block_diffusion_lm_attn_b200 import build
 
@@ -33,15 +40,19 @@ def _compare(o1, l1, o2, l2):
     assert torch.isfinite(o2.float()).all() and torch.isfinite(l2).all()
 
 
+CASES = [
+    # B, Hq, Hkv, b, d, lens, mode
+    (16, 32, 8, 32, 128, [2048] * 16, 0),
+    (8, 32, 8, 28, 128, [513, 4000, 77, 1024, 3001, 900, 12, 2500], 1),
+    (4, 8, 2, 16, 64, [300, 5, 1200, 64], 0),
+    (3, 4, 4, 8, 64, [100, 0, 40], 1),
+]
+
+
 def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
     build.build()
     bd.load()
-    cases = [
-        # B, Hq, Hkv, b, d, lens, mode
-        (16, 32, 8, 32, 128, [2048] * 16, 0),
-        (8, 32, 8, 28, 128, [513, 4000, 77, 1024, 3001, 900, 12, 2500], 1),
-    ]
-    for B, Hq, Hkv, b, d, lens, mode in cases:
+    for B, Hq, Hkv, b, d, lens, mode in CASES:
         S_cap = max(lens) + b
         assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) <= SCRATCH_MAX
         q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
@@ -62,3 +73,57 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
     st = bd.bd_attn_decode_noalloc(A, A, A, A, A, A, B, Hq, Hkv, b, d, 0,
                                    None, S_cap)
     assert st == bd.BD_ERR_UNSUPPORTED
+
+
+def test_noalloc_decode_matches_the_oracle():
+    build.build()
+    bd.load()
+    B, Hq, Hkv, b, d, lens, mode = 4, 8, 2, 28, 128, [700, 2047, 0, 129], 1
+    S_cap = max(lens) + b
+    q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
+                                            cache_len=lens, seed=3)
+    out = torch.empty((B, Hq, b, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, Hq, b), device="cuda")
+    assert _call_noalloc(q.cuda(), kc.cuda(), vc.cuda(), cl.cuda(), mode,
+                         out, lse) == bd.BD_OK
+    torch.cuda.synchronize()
+    assert bd.device_status() == bd.BD_OK
+    ro, rl = oracle.decode(q, kc, vc, cl, mode, 1 / math.sqrt(d))
+    err = np.abs(out.float().cpu().numpy() - ro)
+    assert err.max() <= OUT_MAX and err.mean() <= OUT_MEAN
+    assert np.abs(lse.cpu().numpy() - rl).max() <= LSE_MAX
+
+
+def test_noalloc_decode_inside_a_graph_capture():
+    """After one ordinary call (which looks up the array's address), the
+    entry point can be recorded in a CUDA graph captured in global mode; the
+    replays read the current inputs and match bd_attn_decode."""
+    build.build()
+    bd.load()
+    B, Hq, Hkv, b, d, mode = 8, 32, 8, 32, 128, 0
+    lens = [1500, 900, 2000, 64, 1999, 3, 777, 1024]
+    S_cap = max(lens) + b
+    q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
+                                            cache_len=lens, seed=17)
+    q, kc, vc, cl = q.cuda(), kc.cuda(), vc.cuda(), cl.cuda()
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, b), device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        assert _call_noalloc(q, kc, vc, cl, mode, out, lse) == bd.BD_OK
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, capture_error_mode="global"):
+        assert _call_noalloc(q, kc, vc, cl, mode, out, lse) == bd.BD_OK
+    for seed in (18, 19):
+        q2, _, _, _ = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
+                                              cache_len=lens, seed=seed)
+        q.copy_(q2.cuda())
+        graph.replay()
+        torch.cuda.synchronize()
+        ref_o, ref_l = bd.decode(q, kc, vc, cl, mode)
+        torch.cuda.synchronize()
+        _compare(ref_o, ref_l, out, lse)
+    assert bd.device_status() == bd.BD_OK
