@@ -52,15 +52,36 @@ def flush_l2(flush, i):
                                  device=flush.device)
     torch.sum(_flush_read)
 HOST_COVER_CYCLES = 400000  # ~0.2 ms GPU sleep queued before each timed step
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the dominant
-# kernel, from the ncu captures summarised under profiles/
-# (bd_tc_pair_kernel_fwd_training_shape.md: 201,509,376 read + 100,790,528
-# written; bd_tc_persist_kernel_decode.md: 543,351,040 read + 7,544,064
-# written by the denoising-decode attention kernel, whose combine launch
-# moves no tile data in whole-unit mode).  Set back to None whenever the
-# kernel changes after those counters were taken.
-FWD_TRAFFIC_BYTES = 302299904
-DECODE_TRAFFIC_BYTES = 550895104
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# each dominant kernel, from an ncu capture of the bench's own workload.  Each
+# entry records the SHA-256 (first 16 hex digits) of the kernel sources it was
+# captured with; if the sources differ now, the figure no longer describes the
+# kernel and the bench reports traffic as null.
+KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
+                  "attn_mma.cuh", "bd_common.cuh")
+TRAFFIC = {
+    # kernel: (bytes per launch, source digest at capture time, capture)
+    "bd_tc_pair_kernel": (None, None, None),
+    "bd_tc_persist_kernel<1>": (None, None, None),
+}
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_diffusion_lm_attn_b200", "csrc")
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_of(kernel: str):
+    nbytes, digest, _ = TRAFFIC.get(kernel, (None, None, None))
+    if nbytes is None or digest != kernel_source_digest():
+        return None
+    return nbytes
 
 
 def fwd_flops(s) -> int:
@@ -336,10 +357,16 @@ def run_ours(args):
                 dec_roof = {"bound": "hbm", "achieved": round(gbs, 1),
                             "peak": hbm, "unit": "GB/s",
                             "frac": round(gbs / hbm, 4),
-                            "traffic": DECODE_TRAFFIC_BYTES,
+                            "traffic": traffic_of("bd_tc_persist_kernel<1>"),
                             "peak_source": peak_kind,
                             "kernels": "stream-K attention + combine"}
             del qd, kcd, vcd, o, ls, ws
+    # ---- the rest of the path: backward, cross-attention decode, SPRINT,
+    # speculative append (one call each per step, timed the same way)
+    if only == "all" and not args.quick:
+        n = max(5, args.steps // 10)
+        rows.update(extra_rows(bd, dev, flush, world, sampler, n, hbm,
+                               tf_burst))
     clocks = sampler.stop()
 
     result = None
@@ -364,22 +391,122 @@ def run_ours(args):
                 "bound": "tensor", "achieved": round(fwd_kernel_tflops, 2),
                 "peak": tf_burst, "unit": "TFLOP/s",
                 "frac": round(fwd_kernel_tflops / tf_burst, 4),
-                "traffic": FWD_TRAFFIC_BYTES,
+                "traffic": traffic_of("bd_tc_pair_kernel"),
                 "peak_source": peak_kind + " bf16 burst"},
             "roofline_decode": dec_roof,
             "e2e": e2e,
             "gpu_launches": n_launch,
+            "fwd_kernel": {2: "bd_tc_pair_kernel", 1: "bd_tc_persist_kernel<0>",
+                           0: "bd_mma_attn_kernel"}.get(
+                               bd.bd_attn_debug_fwd_kernel(s.Hq, s.Hkv, s.d)),
             "clocks": clocks,
             "rows": rows,
         }
         if world == 1 and only == "all" and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(s, budget_s=args.cpu_seconds)
+            if not args.quick:
+                result["cpu_baseline_rows"] = {
+                    sd.name: cpu_baseline_decode(sd)
+                    for sd in (bd_inputs.DEC_DENOISE, bd_inputs.DEC_VERIFY)}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if result is not None:
         print(json.dumps(result), flush=True)
+
+
+def extra_rows(bd, dev, flush, world, sampler, n, hbm, tf_burst):
+    """Rows for the backward, cross-attention-only decode, sparse prefix
+    retention and the speculative accept/append step."""
+    rows = {}
+    # backward on the training shape: 5 products per visible pair (S, dP,
+    # dV, dK, dQ) = 2.5 x the forward's FLOPs; three kernels per call
+    s = bd_inputs.FWD_TRAIN
+    q, k, v = bd_inputs.fwd_inputs_for(s)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    g = torch.Generator("cpu").manual_seed(1)
+    dod = torch.randn(q.shape, generator=g).to(torch.bfloat16).to(dev)
+    out, lse = bd.fwd(qd, kd, vd, s.L, s.b, s.scale)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(bd.bd_attn_bwd_workspace_bytes(s.B, s.Hq, s.L),
+                     dtype=torch.uint8, device=dev)
+    t = timed_steps(lambda: bd.bwd(qd, kd, vd, out, lse, dod, s.L, s.b, s.scale,
+                                   dq=dq, dk=dk, dv=dv, workspace=ws),
+                    n, 3, flush, world, sampler) / n
+    tf = 2.5 * fwd_flops(s) / (t * 1e-3) / 1e12
+    rows["bwd_train"] = {"tflops": round(tf, 2), "ms": round(t, 4),
+                         "frac_of_measured_bf16": round(tf / tf_burst, 4),
+                         "kernels": "row pass + dK/dV pass + dQ pass"}
+    del qd, kd, vd, dod, out, lse, dq, dk, dv, ws
+
+    # cross-attention-only decode (mode 2): the denoising shape's canvas of
+    # b = 32 rows over an 8192-token encoder cache
+    sd = bd_inputs.DEC_DENOISE
+    qb, kc, vc, cl = bd_inputs.decode_inputs_for(sd)
+    qd, kcd, vcd, cld = qb.to(dev), kc.to(dev), vc.to(dev), cl.to(dev)
+    o = torch.empty_like(qd)
+    ls = torch.empty((sd.B, sd.Hq, sd.b), device=dev, dtype=torch.float32)
+    wsd = torch.empty(bd.workspace_bytes(sd.B, sd.Hq, sd.Hkv, sd.b, sd.d, sd.S_cap),
+                      dtype=torch.uint8, device=dev)
+    t = timed_steps(lambda: bd.decode(qd, kcd, vcd, cld, 2, out=o, lse=ls,
+                                      workspace=wsd),
+                    n, 3, flush, world, sampler) / n
+    nbytes = (sum(sd.Hkv * int(x) * sd.d * 2 * 2 for x in cl.tolist()) +
+              sd.B * sd.Hq * sd.b * (sd.d * 2 * 2 + 4))
+    gbs = nbytes / (t * 1e-3) / 1e9
+    rows["decode_cross"] = {"gbs": round(gbs, 1), "ms": round(t, 4), "bytes": nbytes,
+                            "frac_of_measured_hbm": round(gbs / hbm, 4)}
+
+    # sparse prefix retention of the same cache: 3/4 image tokens then text,
+    # keep 0.8 of the image and all the text (alpha 0.5)
+    conf = torch.rand((sd.B, sd.S_cap), generator=g).to(dev)
+    mod = torch.zeros((sd.B, sd.S_cap), dtype=torch.uint8)
+    mod[:, :6144] = 1
+    mod = mod.to(dev)
+    ko, vo = torch.empty_like(kcd), torch.empty_like(vcd)
+    wss = torch.empty(bd.bd_sprint_workspace_bytes(sd.B, sd.S_cap),
+                      dtype=torch.uint8, device=dev)
+    res = {}
+
+    def prune():
+        res["r"] = bd.sprint_prune(kcd, vcd, cld, conf, mod, 0.5, 1.0, 0.8,
+                                   k_out=ko, v_out=vo, workspace=wss)
+    t = timed_steps(prune, n, 3, flush, world, sampler) / n
+    kept = int(res["r"][3].sum())
+    row_bytes = sd.Hkv * sd.d * 2
+    nbytes = (sum(int(x) for x in cl.tolist()) * row_bytes  # K read for the norms
+              + kept * row_bytes * 2 * 2)                    # K, V kept: read + write
+    gbs = nbytes / (t * 1e-3) / 1e9
+    rows["sprint_prune"] = {"gbs": round(gbs, 1), "ms": round(t, 4), "bytes": nbytes,
+                            "kept_rows": kept,
+                            "frac_of_measured_hbm": round(gbs / hbm, 4)}
+    del qd, kcd, vcd, o, ls, wsd, ko, vo, wss
+
+    # speculative step bookkeeping of the verification shape (B = 64, b = 28):
+    # accepted length from draft/target tokens, then append the accepted
+    # rows of the block's K/V to the cache (latency-bound)
+    sv = bd_inputs.DEC_VERIFY
+    kc = torch.zeros((sv.B, sv.Hkv, sv.S_cap, sv.d), dtype=torch.bfloat16, device=dev)
+    vc = torch.zeros_like(kc)
+    kn = torch.randn((sv.B, sv.Hkv, sv.b, sv.d), generator=g).to(torch.bfloat16).to(dev)
+    vn = torch.randn((sv.B, sv.Hkv, sv.b, sv.d), generator=g).to(torch.bfloat16).to(dev)
+    draft = torch.randint(0, 4, (sv.B, sv.b), generator=g, dtype=torch.int32).to(dev)
+    target = draft.clone()
+    target[:, sv.b // 2] += 1
+    lens0 = torch.full((sv.B,), 4096, dtype=torch.int32, device=dev)
+    lens = lens0.clone()
+    nacc = torch.empty(sv.B, dtype=torch.int32, device=dev)
+
+    def step():
+        lens.copy_(lens0)
+        bd.spec_accept(draft, target, n_accept=nacc)
+        bd.cache_append(kc, vc, lens, nacc, kn, vn)
+    t = timed_steps(step, n, 3, flush, world, sampler) / n
+    rows["spec_accept_append"] = {"us": round(t * 1e3, 2),
+                                  "rows_appended": int(nacc.sum()) * sv.Hkv,
+                                  "kernels": "copy of lens + accept + append"}
+    return rows
 
 
 # ---------------------------------------------------------------------------
@@ -419,6 +546,30 @@ def cpu_baseline(s, budget_s=15.0, rows_per_step=None, steps=1, warmup=0):
             "sample": "%d seeded query rows of the training shape (of %d), "
                       "fp64, %.2f s per pass" % (len(rows), total, dt),
             "seconds_per_step": dt}
+
+
+def cpu_baseline_decode(sd, budget_s=8.0):
+    """The oracle on a seeded row sample of a block-decode workload.  The
+    oracle gathers each row's keys itself, so its rate is stated as the
+    workload's algorithmic bytes over the time the whole workload would take
+    at the sampled rows' pace (time x total rows / sampled rows)."""
+    import oracle
+    q, kc, vc, cl = bd_inputs.decode_inputs_for(sd)
+    total = sd.B * sd.Hq * sd.b
+    probe = bd_inputs.sample_rows(total, 0, 16, seed=7)
+    t0 = time.perf_counter()
+    oracle.decode(q, kc, vc, cl, sd.mode, sd.scale, rows=probe)
+    dt = time.perf_counter() - t0
+    n = max(16, min(total, int(len(probe) * budget_s / max(dt, 1e-3))))
+    rows = bd_inputs.sample_rows(total, 0, n, seed=11)
+    t0 = time.perf_counter()
+    oracle.decode(q, kc, vc, cl, sd.mode, sd.scale, rows=rows)
+    dt = time.perf_counter() - t0
+    full_s = dt * total / len(rows)
+    return {"value": round(decode_bytes(sd, cl.tolist()) / full_s / 1e9, 4),
+            "unit": "GB/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": "%d seeded query rows of %s (of %d), fp64, %.2f s; rate "
+                      "scaled to the whole workload" % (len(rows), sd.name, total, dt)}
 
 
 def run_reference(args):

@@ -164,6 +164,15 @@ def bd_attn_debug_inject_fault(kind):
     return fn(kind)
 
 
+def bd_attn_debug_fwd_kernel(Hq, Hkv, d):
+    """Test hook (include/bd_attn_debug.h): which forward kernel runs for
+    these sizes (2 paired tcgen05, 1 one-tile tcgen05, 0 mma.sync, -1 none)."""
+    fn = load().bd_attn_debug_fwd_kernel
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int] * 3
+    return fn(Hq, Hkv, d)
+
+
 def bd_attn_debug_set_grid(ctas):
     """Test hook (include/bd_attn_debug.h): cap the grid of the persistent
     head-dim-128 kernels at `ctas` CTAs (0 restores one CTA per SM)."""

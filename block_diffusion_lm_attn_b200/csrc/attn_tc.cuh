@@ -213,6 +213,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
           "=r"(r[30]), "=r"(r[31])
         : "r"(taddr));
 }
+// 32 lanes x 16 columns -> 16 registers per thread
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+          "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+          "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
 {
     asm volatile(
@@ -369,6 +381,37 @@ __device__ __forceinline__ void softmax_p_tile(const float *s, float sl2,
     }
 }
 
+// As softmax_p_tile for a tile in which only the 32-column words set in
+// `live` (the same for every lane of the warp) hold a visible key for some row
+// of the warp: the other words get P = 0 without any exponential.
+__device__ __forceinline__ void softmax_p_tile_live(const float *s, float sl2,
+                                                    float nm, uint32_t ts,
+                                                    float *rsum, uint32_t live)
+{
+#pragma unroll
+    for (int c4 = 0; c4 < kTcN / 32; ++c4) {
+        uint32_t pk[16];
+        if ((live >> c4) & 1u) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+                float x0, x1;
+                const int b0 = c4 * 32 + c;
+                ffma2(x0, x1, s[b0], s[b0 + 1], sl2, sl2, nm, nm);
+                x0 = ex2(x0);
+                x1 = ex2(x1);
+                const int a = (c >> 1) & 1;
+                fadd2(rsum[2 * a], rsum[2 * a + 1], rsum[2 * a], rsum[2 * a + 1], x0, x1);
+                pk[c / 2] = pack_bf16x2(x0, x1);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = 0u;
+        }
+        tmem_st16(ts + c4 * 16, pk);
+    }
+}
+
 // Bits [a, b) of a 32-bit word, with a and b clamped to [0, 32].
 __device__ __forceinline__ uint32_t range_bits(int a, int b)
 {
@@ -377,6 +420,121 @@ __device__ __forceinline__ uint32_t range_bits(int a, int b)
     const uint32_t below_b = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
     const uint32_t below_a = a >= 32 ? 0xffffffffu : ((1u << a) - 1u);
     return below_b & ~below_a;
+}
+
+} // namespace bd
+
+namespace bd {
+
+// One key tile of the online softmax for the query row of this thread (its
+// TMEM lane), in a warp that holds 32 consecutive rows of a 128-row tile.
+//  - S (128 fp32 columns at TMEM address ts) is read into registers.
+//  - On a PARTIAL tile, columns outside the row's visible intervals
+//    [sp.a0, sp.a1) U [sp.a2, sp.a3), or at or past key khi, become -inf
+//    (ks = first key of the tile); 32-column words that no row of the warp
+//    sees are skipped altogether.
+//  - The running maximum m_used (log2 units) is raised lazily, only when the
+//    tile maximum exceeds it by more than 8; if any lane raises it and
+//    rescale_o is set, the warp waits for the previous PV (wait_prev_pv,
+//    false on abort) and rescales its rows of O (128 fp32 columns at t_o) in
+//    TMEM.
+//  - P = 2^(s * sl2 - m_used) is written as bf16 over S, its sum added to l.
+// Returns false if wait_prev_pv failed.  The caller waits for the TMEM
+// stores and signals P.
+template <bool EMU, typename WaitPV>
+__device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool full,
+                                             const Span &sp, int ks, int khi,
+                                             float sl2, bool rescale_o,
+                                             float &m_used, float &l,
+                                             WaitPV wait_prev_pv)
+{
+    uint32_t sr[kTcN];
+    tmem_ld32(ts + 0, sr + 0);
+    tmem_ld32(ts + 32, sr + 32);
+    tmem_ld32(ts + 64, sr + 64);
+    tmem_ld32(ts + 96, sr + 96);
+    tmem_wait_ld();
+    float s[kTcN];
+#pragma unroll
+    for (int c = 0; c < kTcN; ++c)
+        s[c] = __uint_as_float(sr[c]);
+    uint32_t live = 0xFu;
+    if (!full) {
+        const int e = min(khi, ks + kTcN);
+        const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
+        const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
+        live = 0u;
+#pragma unroll
+        for (int w = 0; w < kTcN / 32; ++w) {
+            const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                               range_bits(lo1 - 32 * w, hi1 - 32 * w);
+            live |= (__any_sync(0xffffffffu, m != 0u) ? 1u : 0u) << w;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+                s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
+        }
+    }
+    float mc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        mc[i] = -INFINITY;
+    if (live == 0xFu) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            mc[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+        for (int c = 16; c < kTcN; c += 16)
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
+    } else {
+#pragma unroll
+        for (int w = 0; w < kTcN / 32; ++w) {
+            if ((live >> w) & 1u) {
+#pragma unroll
+                for (int c = 32 * w; c < 32 * w + 32; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
+            }
+        }
+    }
+    const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
+                           fmaxf(mc[6], mc[7]));
+    const float mt = mx * sl2;
+    // the TMEM read-modify-write of O is warp-collective, so the warp takes
+    // it if any lane needs it (with factor 1 on the others)
+    const bool need = mt > m_used + 8.f;
+    const bool warp_need = __any_sync(0xffffffffu, need);
+    float c = 1.f;
+    if (need) {
+        c = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
+        l *= c;
+        m_used = mt;
+    }
+    if (rescale_o && warp_need) {
+        if (!__all_sync(0xffffffffu, wait_prev_pv()))
+            return false;
+        tc_fence_after();
+#pragma unroll
+        for (int q8 = 0; q8 < kTcD / 16; ++q8) {
+            uint32_t o[16];
+            tmem_ld16(t_o + q8 * 16, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                o[i] = __float_as_uint(__uint_as_float(o[i]) * c);
+            tmem_st16(t_o + q8 * 16, o);
+        }
+    }
+    const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
+    float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+    if (live == 0xFu)
+        softmax_p_tile<EMU>(s, sl2, nm, ts, rsum);
+    else
+        softmax_p_tile_live(s, sl2, nm, ts, rsum, live);
+    l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+    return true;
 }
 
 } // namespace bd

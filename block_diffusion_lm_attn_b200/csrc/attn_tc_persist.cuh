@@ -562,79 +562,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (!ok)
                     break;
                 tc_fence_after();
-                const uint32_t ts = t_s0 + (uint32_t)sb * 128 + lane_off;
-                uint32_t sr[128];
-                tmem_ld32(ts + 0, sr + 0);
-                tmem_ld32(ts + 32, sr + 32);
-                tmem_ld32(ts + 64, sr + 64);
-                tmem_ld32(ts + 96, sr + 96);
-                tmem_wait_ld();
-                float s[kTcN];
-#pragma unroll
-                for (int c = 0; c < kTcN; ++c)
-                    s[c] = __uint_as_float(sr[c]);
                 const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
-                if (!full) {
-                    const int e = min(khi, ks + kTcN);
-                    const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
-                    const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
-#pragma unroll
-                    for (int w = 0; w < kTcN / 32; ++w) {
-                        const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
-                                           range_bits(lo1 - 32 * w, hi1 - 32 * w);
-#pragma unroll
-                        for (int c = 0; c < 32; ++c)
-                            s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
-                    }
-                }
-                float mc[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    mc[i] = fmaxf(s[i], s[8 + i]);
-#pragma unroll
-                for (int c = 16; c < kTcN; c += 16)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
-                const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]),
-                                       fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
-                const float mt = mx * sl2;
-                // lazy rescale (threshold 2^8); the TMEM read-modify-write of O
-                // is warp-collective, so the warp takes it if any lane needs it
-                const bool need = mt > m_used + 8.f;
-                const bool warp_need = __any_sync(0xffffffffu, need);
-                float c = 1.f;
-                if (need) {
-                    c = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
-                    l *= c;
-                    m_used = mt;
-                }
-                if (jj >= 1 && warp_need) {
-                    const long long jp = jg - 1; // PV_{jp} done => O stable
-                    ok = __all_sync(0xffffffffu,
-                                    mbar_wait(bar_odone0 + 8 * (jp & 1),
-                                              (uint32_t)((jp >> 1) & 1), abort_flag));
-                    if (!ok)
-                        break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int q4 = 0; q4 < kTcD / 32; ++q4) {
-                        uint32_t o[32];
-                        tmem_ld32(t_o + lane_off + q4 * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * c);
-                        tmem_st32(t_o + lane_off + q4 * 32, o);
-                    }
-                }
-                const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
-                float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+                const long long jp = jg - 1; // PV_{jp} done => O stable
                 // the FMA-pipe exponential relieves the special-function
                 // unit where the softmax paces the tensor pipe (forward); the
                 // HBM-bound decode measured faster without it
-                softmax_p_tile<KIND == 0 && kEmuExp2>(s, sl2, nm, ts, rsum);
-                l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+                ok = softmax_tile<KIND == 0 && kEmuExp2>(
+                    t_s0 + (uint32_t)sb * 128 + lane_off, t_o + lane_off, full, sp, ks, khi, sl2,
+                    jj >= 1, m_used, l, [&] {
+                        return mbar_wait(bar_odone0 + 8 * (jp & 1), (uint32_t)((jp >> 1) & 1),
+                                         abort_flag);
+                    });
+                if (!ok)
+                    break;
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(bar_pfull0 + 8 * sb);

@@ -56,7 +56,8 @@ bool pair_kernel_usable()
         cudaFuncAttributes a;
         u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel) == cudaSuccess &&
              (long long)a.numRegs * bd::kPairThreads >=
-                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther)
+                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther +
+                     128LL * bd::kPairRegsEpi)
                 ? 1
                 : 0;
         usable.store(u);
@@ -127,7 +128,11 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
     return true;
 }
 
-// Per-device cache of the internal decode workspace (workspace == NULL).
+// Per-device internal decode workspace (workspace == NULL).  A buffer once
+// handed out is never freed: a CUDA graph captured earlier may still hold
+// its address.  When a call needs more, a larger buffer is allocated and
+// becomes the current one; the smaller ones stay allocated (and valid for
+// the graphs that recorded them) until the process exits.
 struct InternalWorkspace {
     std::mutex mu;
     void *ptr[64] = {};
@@ -142,14 +147,10 @@ bd_status get_internal_workspace(size_t need, void **out)
         return BD_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_ws.mu);
     if (g_ws.bytes[dev] < need) {
-        if (g_ws.ptr[dev])
-            cudaFree(g_ws.ptr[dev]);
-        g_ws.ptr[dev] = nullptr;
-        g_ws.bytes[dev] = 0;
-        if (cudaMalloc(&g_ws.ptr[dev], need) != cudaSuccess) {
-            g_ws.ptr[dev] = nullptr;
+        void *p = nullptr;
+        if (cudaMalloc(&p, need) != cudaSuccess)
             return BD_ERR_CUDA;
-        }
+        g_ws.ptr[dev] = p; // the previous buffer is kept, not freed
         g_ws.bytes[dev] = need;
     }
     *out = g_ws.ptr[dev];
@@ -686,6 +687,15 @@ bd_status bd_attn_debug_inject_fault(int kind)
     return cudaMemcpyToSymbol(bd::g_fault_skip_k, &kind, sizeof kind) == cudaSuccess
                ? BD_OK
                : BD_ERR_CUDA;
+}
+
+int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d)
+{
+    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !supported_d(d))
+        return -1;
+    if (d != 128)
+        return 0;
+    return ((Hq / Hkv) % 2 == 0 && pair_kernel_usable()) ? 2 : 1;
 }
 
 bd_status bd_attn_debug_set_grid(int ctas)

@@ -167,9 +167,16 @@ BD_API size_t bd_attn_bwd_workspace_bytes(int B, int Hq, int L);
  *                    bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap)
  *                    bytes, 256-byte aligned, used for the split-KV partial
  *                    results; its contents on entry do not matter.  NULL
- *                    makes the library use a buffer it allocates once per
- *                    device and keeps (that first call allocates, so it must
- *                    not be inside a stream capture).
+ *                    makes the library use an internal buffer of the current
+ *                    device: a call that needs more than the current one
+ *                    allocates a larger buffer (so that call must not be
+ *                    inside a stream capture); buffers handed out are never
+ *                    freed, so graphs captured with an earlier one stay
+ *                    valid.  Every NULL-workspace call on a device shares
+ *                    the current buffer: calls whose kernels may overlap on
+ *                    the GPU (two streams without ordering between them)
+ *                    race on it and give wrong results -- order them, or
+ *                    pass each stream its own workspace.
  *
  * Errors: BD_ERR_INVALID_ARG for a null or misaligned pointer, any size <= 0,
  * Hq % Hkv != 0, S_cap < b in modes 0 and 1, intra_block_mode not 0/1/2, or

@@ -87,6 +87,18 @@ FWD_GRID = [
 ]
 
 
+def test_fwd_kernel_selection():
+    """Even GQA groups of head dim 128 run the paired tcgen05 kernel (the
+    one the benchmark times), odd groups the one-tile tcgen05 kernel, head
+    dims 32 and 64 the mma.sync kernel; so the grid below covers each."""
+    assert bd.bd_attn_debug_fwd_kernel(32, 8, 128) == 2
+    assert bd.bd_attn_debug_fwd_kernel(4, 2, 128) == 2
+    assert bd.bd_attn_debug_fwd_kernel(8, 8, 128) == 1
+    assert bd.bd_attn_debug_fwd_kernel(3, 1, 128) == 1
+    assert bd.bd_attn_debug_fwd_kernel(2, 2, 64) == 0
+    assert bd.bd_attn_debug_fwd_kernel(3, 2, 128) == -1
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,L,b,d", FWD_GRID)
 def test_fwd_grid_all_elements(B, Hq, Hkv, L, b, d):
     q, k, v = bd_inputs.fwd_inputs(B, Hq, Hkv, L, d, seed=L + b + d)
@@ -265,3 +277,40 @@ def test_decode_bad_cache_len_is_reported():
     assert torch.isnan(lse[1]).all() and torch.isfinite(lse[0]).all()
     ro, rl = oracle.decode(q[:1], kc[:1], vc[:1], [10], 0, 1 / math.sqrt(d))
     check(out[:1], lse[:1], ro, rl, "good sequence next to a bad one")
+
+
+def test_internal_workspace_survives_growth_under_a_captured_graph():
+    """A graph captured with the library's internal decode workspace
+    (workspace = NULL) stays valid after a later call needs a larger
+    internal workspace: the earlier buffer is kept, not freed."""
+    B, Hq, Hkv, b, d = 4, 32, 8, 32, 128
+    lens = [900, 17, 2048, 511]
+    S_cap = 2100
+    q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
+                                            cache_len=lens, seed=23)
+    qd, kd, vd, cd = q.cuda(), kc.cuda(), vc.cuda(), cl.cuda()
+    out = torch.empty_like(qd)
+    lse = torch.empty((B, Hq, b), device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        bd.decode(qd, kd, vd, cd, 0, out=out, lse=lse, stream=s)  # allocates
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            bd.decode(qd, kd, vd, cd, 0, out=out, lse=lse, stream=s)
+    torch.cuda.synchronize()
+    # a head-dim-64 call whose split-KV scratch exceeds the current buffer
+    B2, Hq2, Hkv2, b2, d2 = 128, 32, 8, 32, 64
+    assert (bd.workspace_bytes(B2, Hq2, Hkv2, b2, d2, 64) >
+            bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap))
+    q2, kc2, vc2, cl2 = bd_inputs.decode_inputs(B2, Hq2, Hkv2, b2, d2, 64,
+                                                cache_len=[20] * B2, seed=24)
+    bd.decode(q2.cuda(), kc2.cuda(), vc2.cuda(), cl2.cuda(), 1)
+    torch.cuda.synchronize()
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert bd.device_status() == bd.BD_OK
+    ro, rl = oracle.decode(q, kc, vc, cl, 0, 1 / math.sqrt(d))
+    check(out, lse, ro, rl, "graph replay after workspace growth")
