@@ -316,14 +316,16 @@ def run_ours(args):
         del qd, kd, vd, out, lse
 
     # ---- long-context block-size sweep
-    if only == "all" and not args.quick:
+    if (only == "all" and not args.quick) or only == "fwd_long":
         for bb, sl in sorted(bd_inputs.FWD_LONG.items()):
+            if only == "fwd_long" and bb != 64:
+                continue
             q, k, v = bd_inputs.fwd_inputs_for(sl)
             qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
             o = torch.empty_like(qd)
             ls = torch.empty((sl.B, sl.Hq, 2 * sl.L), device=dev,
                              dtype=torch.float32)
-            n = max(5, args.steps // 10)
+            n = max(5, args.steps // 10) if only == "all" else args.steps
             t = timed_steps(lambda: bd.fwd(qd, kd, vd, sl.L, sl.b, sl.scale,
                                            out=o, lse=ls),
                             n, 3, flush, world, sampler) / n
@@ -363,8 +365,8 @@ def run_ours(args):
             del qd, kcd, vcd, o, ls, ws
     # ---- the rest of the path: backward, cross-attention decode, SPRINT,
     # speculative append (one call each per step, timed the same way)
-    if only == "all" and not args.quick:
-        n = max(5, args.steps // 10)
+    if (only == "all" and not args.quick) or only == "extra":
+        n = max(5, args.steps // 10) if only == "all" else args.steps
         rows.update(extra_rows(bd, dev, flush, world, sampler, n, hbm,
                                tf_burst))
     clocks = sampler.stop()
@@ -611,8 +613,11 @@ def main():
                     help="skip the long-context sweep")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--only", choices=["all", "fwd", "decode"], default="all",
-                    help="time only the training-shape fwd or only decode "
+    ap.add_argument("--only", choices=["all", "fwd", "decode", "fwd_long",
+                                       "extra"], default="all",
+                    help="time only the training-shape fwd, only decode, only "
+                         "the long-context fwd with b=64, or only the "
+                         "backward / cross-decode / SPRINT / append rows "
                          "(used for profiling captures)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps

@@ -207,9 +207,9 @@ __global__ void __launch_bounds__(kSelThreads)
 {
     __shared__ double red_d[32];
     __shared__ int red_i[32];
-    __shared__ unsigned int hist[256];
-    __shared__ unsigned long long s_prefix;
-    __shared__ int s_need;
+    __shared__ unsigned int hist[512];
+    __shared__ unsigned long long s_prefix[2];
+    __shared__ int s_need[2], s_want[2];
     const int i = blockIdx.x;
     const int len = cache_len[i];
     const int tid = threadIdx.x;
@@ -241,59 +241,88 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
 
     // kept flags live in the kept row itself until the final compaction:
-    // 1 = kept, 0 = dropped
-    for (int m = 0; m < 2; ++m) {
-        int cnt = 0;
-        for (int p = p0; p < p1; ++p)
-            cnt += ((modality[row + p] != 0) == m);
-        const int n_m = block_sum(cnt, red_i);
-        const double r = m == 0 ? keep_text : keep_image;
-        long long want = (long long)floor(r * (double)n_m + 0.5);
-        want = max(0LL, min(want, (long long)n_m));
-        // radix select of the want-th largest key among this modality
-        if (tid == 0) {
-            s_prefix = 0;
-            s_need = (int)want; // rank still to find inside the prefix
+    // 1 = kept, 0 = dropped.  Both modalities are selected together: an
+    // 8-pass radix select (8 bits per pass) of each modality's want-th
+    // largest score key, one 256-bin histogram per modality.
+    {
+        int cnt1 = 0, cnt = 0;
+        for (int p = p0; p < p1; ++p) {
+            cnt1 += modality[row + p] != 0;
+            ++cnt;
         }
-        __syncthreads();
-        if (want > 0) {
-            for (int pass = 0; pass < 8; ++pass) {
-                const int shift = 56 - 8 * pass;
-                for (int k = tid; k < 256; k += blockDim.x)
-                    hist[k] = 0;
-                __syncthreads();
-                const unsigned long long pre = s_prefix;
-                const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
-                for (int p = p0; p < p1; ++p) {
-                    if ((modality[row + p] != 0) != m)
-                        continue;
-                    const unsigned long long key = dkey(score[row + p]);
-                    if ((key & hmask) == pre)
-                        atomicAdd(&hist[(key >> shift) & 255], 1u);
-                }
-                __syncthreads();
-                if (tid == 0) {
-                    int need = s_need;
-                    int dgt = 255;
-                    for (; dgt > 0; --dgt) {
-                        if ((int)hist[dgt] >= need)
-                            break;
-                        need -= (int)hist[dgt];
-                    }
-                    s_prefix = pre | ((unsigned long long)dgt << shift);
-                    s_need = need;
-                }
-                __syncthreads();
+        const int n_img = block_sum(cnt1, red_i);
+        const int n_all = block_sum(cnt, red_i);
+        if (tid == 0) {
+            const int n_m[2] = {n_all - n_img, n_img};
+            for (int m = 0; m < 2; ++m) {
+                const double r = m == 0 ? keep_text : keep_image;
+                long long want = (long long)floor(r * (double)n_m[m] + 0.5);
+                want = max(0LL, min(want, (long long)n_m[m]));
+                s_want[m] = (int)want;
+                s_need[m] = (int)want; // rank still to find below the prefix
+                s_prefix[m] = 0;
             }
         }
+        __syncthreads();
+    }
+    for (int pass = 0; pass < 8; ++pass) {
+        const int shift = 56 - 8 * pass;
+        for (int k = tid; k < 512; k += blockDim.x)
+            hist[k] = 0;
+        __syncthreads();
+        const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
+        const unsigned long long pre0 = s_prefix[0], pre1 = s_prefix[1];
+        for (int p = p0; p < p1; ++p) {
+            const int m = modality[row + p] != 0;
+            const unsigned long long key = dkey(score[row + p]);
+            if ((key & hmask) == (m ? pre1 : pre0))
+                atomicAdd(&hist[m * 256 + ((key >> shift) & 255)], 1u);
+        }
+        __syncthreads();
+        // warp m finds the digit of modality m: lane l owns the 8 digits
+        // 255 - 8 l .. 248 - 8 l, scanned from the top
+        const int w = tid >> 5, lane = tid & 31;
+        if (w < 2 && s_want[w] > 0) {
+            const unsigned int *hm = hist + w * 256;
+            int sum = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                sum += (int)hm[255 - 8 * lane - u];
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o)
+                    incl += y;
+            }
+            const int need = s_need[w];
+            const unsigned int hit = __ballot_sync(0xffffffffu, incl >= need);
+            // need >= 1 and the modality's candidates number at least need,
+            // so some lane holds the target
+            const int tl = __ffs(hit) - 1;
+            if (lane == tl) {
+                int rem = need - (incl - sum);
+                int dgt = 255 - 8 * lane;
+                for (int u = 0; u < 7; ++u, --dgt) {
+                    if ((int)hm[dgt] >= rem)
+                        break;
+                    rem -= (int)hm[dgt];
+                }
+                s_prefix[w] |= (unsigned long long)dgt << shift;
+                s_need[w] = rem;
+            }
+        }
+        __syncthreads();
+    }
+    for (int m = 0; m < 2; ++m) {
         // keys above the threshold are kept; of the keys equal to it, the
         // s_need lowest positions
-        const unsigned long long thr = s_prefix;
-        const int need_eq = want > 0 ? s_need : 0;
+        const bool any = s_want[m] > 0;
+        const unsigned long long thr = s_prefix[m];
+        const int need_eq = any ? s_need[m] : 0;
         int eq = 0;
         for (int p = p0; p < p1; ++p)
-            if ((modality[row + p] != 0) == m && want > 0 &&
-                dkey(score[row + p]) == thr)
+            if ((modality[row + p] != 0) == m && any && dkey(score[row + p]) == thr)
                 ++eq;
         int tot_eq;
         int before = block_scan_excl(eq, red_i, tot_eq);
@@ -301,7 +330,7 @@ __global__ void __launch_bounds__(kSelThreads)
             if ((modality[row + p] != 0) != m)
                 continue;
             int keep = 0;
-            if (want > 0) {
+            if (any) {
                 const unsigned long long key = dkey(score[row + p]);
                 if (key > thr)
                     keep = 1;
