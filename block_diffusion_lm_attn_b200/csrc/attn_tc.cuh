@@ -431,8 +431,8 @@ namespace bd {
 //  - S (128 fp32 columns at TMEM address ts) is read into registers.
 //  - On a PARTIAL tile, columns outside the row's visible intervals
 //    [sp.a0, sp.a1) U [sp.a2, sp.a3), or at or past key khi, become -inf
-//    (ks = first key of the tile); 32-column words that no row of the warp
-//    sees are skipped altogether.
+//    (ks = first key of the tile).  With SKIP, 32-column words that no row of
+//    the warp sees also skip their max and exponentials.
 //  - The running maximum m_used (log2 units) is raised lazily, only when the
 //    tile maximum exceeds it by more than 8; if any lane raises it and
 //    rescale_o is set, the warp waits for the previous PV (wait_prev_pv,
@@ -441,7 +441,7 @@ namespace bd {
 //  - P = 2^(s * sl2 - m_used) is written as bf16 over S, its sum added to l.
 // Returns false if wait_prev_pv failed.  The caller waits for the TMEM
 // stores and signals P.
-template <bool EMU, typename WaitPV>
+template <bool EMU, bool SKIP, typename WaitPV>
 __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool full,
                                              const Span &sp, int ks, int khi,
                                              float sl2, bool rescale_o,
@@ -463,22 +463,21 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
         const int e = min(khi, ks + kTcN);
         const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
         const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
-        live = 0u;
+        if (SKIP)
+            live = 0u;
 #pragma unroll
         for (int w = 0; w < kTcN / 32; ++w) {
             const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
-            live |= (__any_sync(0xffffffffu, m != 0u) ? 1u : 0u) << w;
+            if (SKIP)
+                live |= (__any_sync(0xffffffffu, m != 0u) ? 1u : 0u) << w;
 #pragma unroll
             for (int c = 0; c < 32; ++c)
                 s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
         }
     }
     float mc[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        mc[i] = -INFINITY;
-    if (live == 0xFu) {
+    if (!SKIP || live == 0xFu) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             mc[i] = fmaxf(s[i], s[8 + i]);
@@ -488,6 +487,9 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
             for (int i = 0; i < 8; ++i)
                 mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
     } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            mc[i] = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kTcN / 32; ++w) {
             if ((live >> w) & 1u) {
@@ -517,19 +519,19 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
             return false;
         tc_fence_after();
 #pragma unroll
-        for (int q8 = 0; q8 < kTcD / 16; ++q8) {
-            uint32_t o[16];
-            tmem_ld16(t_o + q8 * 16, o);
+        for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+            uint32_t o[32];
+            tmem_ld32(t_o + q4 * 32, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
+            for (int i = 0; i < 32; ++i)
                 o[i] = __float_as_uint(__uint_as_float(o[i]) * c);
-            tmem_st16(t_o + q8 * 16, o);
+            tmem_st32(t_o + q4 * 32, o);
         }
     }
     const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
     float rsum[4] = {0.f, 0.f, 0.f, 0.f};
-    if (live == 0xFu)
+    if (!SKIP || live == 0xFu)
         softmax_p_tile<EMU>(s, sl2, nm, ts, rsum);
     else
         softmax_p_tile_live(s, sl2, nm, ts, rsum, live);

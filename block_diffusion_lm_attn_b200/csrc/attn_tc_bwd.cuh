@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar_sfull(x), 1);
-            mbar_init(bar_pfull(x), 128);
+            mbar_init(bar_pfull(x), 4); // one arrival per compute warp
         }
         mbar_init(bar_odone, 1);
         mbar_init(bar_ofree, 128);
@@ -505,7 +505,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_st16(t_dp(x) + lane_off + 16, dk + 16);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar_pfull(x));
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_pfull(x));
             }
             if (!ok)
                 break;
@@ -586,8 +588,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar_kvfull = [&](int s) { return bar0 + 16 + 8 * s; };
     auto bar_kvempty = [&](int s) { return bar0 + 32 + 8 * s; };
     const uint32_t bar_sfull = bar0 + 48;  // S, dP ready
-    const uint32_t bar_sfree = bar0 + 56;  // S, dP read into registers (128)
-    auto bar_dsfull = [&](int x) { return bar0 + 64 + 8 * x; };  // (128)
+    const uint32_t bar_sfree = bar0 + 56;  // S, dP read into registers
+    auto bar_dsfull = [&](int x) { return bar0 + 64 + 8 * x; };
     auto bar_dsfree = [&](int x) { return bar0 + 80 + 8 * x; };
     const uint32_t bar_qdone = bar0 + 96;  // the item's last dQ retired
     const uint32_t bar_dqfree = bar0 + 104; // dQ read out (128)
@@ -606,11 +608,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_kvfull(s), 1);
             mbar_init(bar_kvempty(s), 1);
-            mbar_init(bar_dsfull(s), 128);
+            mbar_init(bar_dsfull(s), 4); // one arrival per compute warp
             mbar_init(bar_dsfree(s), 1);
         }
         mbar_init(bar_sfull, 1);
-        mbar_init(bar_sfree, 128);
+        mbar_init(bar_sfree, 4);
         mbar_init(bar_qdone, 1);
         mbar_init(bar_dqfree, 128);
         mbar_init(bar_final, 1);
@@ -849,7 +851,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     tmem_wait_ld();
                     if (h == 1) {
                         tc_fence_before();
-                        mbar_arrive(bar_sfree); // S, dP may be overwritten
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive(bar_sfree); // S, dP may be overwritten
                     }
 #pragma unroll
                     for (int c = 0; c < 64; c += 2) {
@@ -869,7 +873,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(bar_dsfull(x));
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_dsfull(x));
             }
             if (!ok)
                 break;

@@ -9,37 +9,31 @@
 // other's PV and next QK, so each MMA wait covers twice the work of the
 // one-tile kernel and K/V traffic from L2 halves.
 //
-// Roles: warps 0-3 softmax of tile A (thread t = row t = TMEM lane t), warps
-// 4-7 softmax of tile B, warp 8 TMA producer of Q and K (and the work-item
-// fetch), warp 9 MMA issuer, warp 10 TMA producer of V, warp 11 idle, warps
-// 12-15 epilogue: they read each finished O out of tensor memory, normalise
-// it and store it, so the softmax warps go straight on to the next item.
-// setmaxnreg gives most registers to the two softmax warpgroups.
+// Roles: warps 0-3 softmax and epilogue of tile A (thread t = row t = TMEM
+// lane t), warps 4-7 the same for tile B, warp 8 TMA producer of Q and K
+// (and the work-item fetch), warp 9 MMA issuer, warp 10 TMA producer of V,
+// warp 11 idle.  setmaxnreg moves registers from warpgroup 2 to the two
+// softmax warpgroups.
 //
 // TMEM: S_A columns [0, 128), S_B [128, 256), O_A [256, 384), O_B [384, 512);
 // P (bf16) overwrites its own S.  Shared memory: the two Q tiles of the
-// current item (one buffer), two K and two V stages, the epilogue's output
-// staging, each item's row sums and maxima, barriers.
+// current item (one buffer), two K and two V stages, per-warp output
+// staging, barriers.
 //
 // MMA issue order per key tile j (the chains of A and B interleave):
 //   PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1)
 // so QK_A(j+1) overwrites S_A only after PV_A(j) -- which read P_A(j) from
 // it -- was issued (tcgen05.mma from one thread execute in issue order).
-//
-// The Q/K producer takes the next item from the global counter while the
-// current one starts, and prefetches that item's Q tiles into L2, so its
-// later load into the (single) Q buffer is an L2 hit.
 #pragma once
 
 #include "attn_tc_persist.cuh"
 
 namespace bd {
 
-constexpr int kPairThreads = 512;
-constexpr int kPairRegsSoftmax = 160; // setmaxnreg of warpgroups 0 and 1
-constexpr int kPairRegsOther = 104;   // setmaxnreg of warpgroup 2
-constexpr int kPairRegsEpi = 88;      // setmaxnreg of warpgroup 3
-static_assert(128 * (2 * kPairRegsSoftmax + kPairRegsOther + kPairRegsEpi) <=
+constexpr int kPairThreads = 384;
+constexpr int kPairRegsSoftmax = 208; // setmaxnreg of warpgroups 0 and 1
+constexpr int kPairRegsOther = 88;    // setmaxnreg of warpgroup 2
+static_assert(2 * 128 * kPairRegsSoftmax + 128 * kPairRegsOther <=
                   kPairThreads * (65536 / kPairThreads / 8 * 8),
               "register split above the launch's allocation");
 
@@ -47,9 +41,8 @@ static_assert(128 * (2 * kPairRegsSoftmax + kPairRegsOther + kPairRegsEpi) <=
 constexpr int kPairSmemQ = 0;                           // tiles A, B
 constexpr int kPairSmemK = kPairSmemQ + 2 * kTileBytes; // 2 stages
 constexpr int kPairSmemV = kPairSmemK + 2 * kTileBytes; // 2 stages
-constexpr int kPairSmemEpi = kPairSmemV + 2 * kTileBytes; // 4 warps x 4 KB
-constexpr int kPairSmemLM = kPairSmemEpi + 4 * 32 * 128;  // [2][2][2][128] fp32
-constexpr int kPairSmemBar = kPairSmemLM + 2 * 2 * 2 * 128 * 4;
+constexpr int kPairSmemEpi = kPairSmemV + 2 * kTileBytes; // 8 warps x 4 KB
+constexpr int kPairSmemBar = kPairSmemEpi + 8 * 32 * 128;
 constexpr int kPairSmemBytes = kPairSmemBar + 512 + 1024;
 static_assert(kPairSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
@@ -92,15 +85,6 @@ __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
     sg.nt = sg.n0 + n1;
 }
 
-// L2 prefetch of one 64-column box of a tensor map (no shared memory).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *tm, int c0, int c1, int c2)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
 __global__ void __launch_bounds__(kPairThreads, 1)
     bd_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -125,14 +109,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t bar_final = bar0 + 160;
     const uint32_t bar_ifull0 = bar0 + 168;  // 4: work item published
     const uint32_t bar_iempty0 = bar0 + 200; // 4: work item read by all roles
-    auto bar_lfull = [&](int x) { return bar0 + 232 + 8 * x; }; // row sums of O_x
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 256);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 384);
     volatile uint32_t *tmem_slot =
         reinterpret_cast<volatile uint32_t *>(sbase + kPairSmemBar + 392);
-    // row sum l and running maximum m of tile x of item si:
-    // lm[((si & 1) * 2 + x) * 2 + {0: l, 1: m}][row]
-    float *lm = reinterpret_cast<float *>(sbase + kPairSmemLM);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -151,13 +131,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mbar_init(bar_odone(x, 0), 1);
             mbar_init(bar_odone(x, 1), 1);
             mbar_init(bar_ofree(x), 128);
-            mbar_init(bar_lfull(x), 128);
         }
         mbar_init(bar_final, 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_ifull0 + 8 * i, 1);
-            // MMA, V producer, 256 softmax threads, 128 epilogue threads
-            mbar_init(bar_iempty0 + 8 * i, 386);
+            mbar_init(bar_iempty0 + 8 * i, 258); // MMA, V producer, 256 softmax threads
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -174,14 +152,26 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     PairSeg sg;
-    // Next item of a consumer role: published by the Q/K producer in
-    // item_ring[si % 4].
-    auto next_seg = [&](int si, bool &ok) -> bool {
+    // Next item of this CTA, identical for every role: the Q/K producer
+    // takes it from the launch's global counter and publishes it in
+    // item_ring[si % 4]; the other roles read it there.
+    auto next_seg = [&](int si, bool producer, bool &ok) -> bool {
         const int slot = si & 3;
-        if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
-            return false;
-        const int w = item_ring[slot];
-        mbar_arrive(bar_iempty0 + 8 * slot);
+        int w;
+        if (producer) {
+            if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
+                                             (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
+                return false;
+            const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
+            w = (long long)t < pair_items(p) ? (int)t : -1;
+            item_ring[slot] = w;
+            mbar_arrive(bar_ifull0 + 8 * slot);
+        } else {
+            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+                return false;
+            w = item_ring[slot];
+            mbar_arrive(bar_iempty0 + 8 * slot);
+        }
         if (w < 0)
             return false;
         pair_item(p, w, sg);
@@ -191,7 +181,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         return it < sg.n0 ? sg.lo0 + it * kTcN : sg.lo1 + (it - sg.n0) * kTcN;
     };
 
-    if (warp >= 8 && warp < 12) {
+    if (warp >= 8) {
     // warpgroup 2 gives registers to the softmax warpgroups; every warp of
     // it executes this one instruction
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsOther));
@@ -199,32 +189,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // ---------------------------------------- TMA producer: Q and K
         if (lane == 0) {
             bool ok = true;
-            long long g = 0, kiss = 0;
-            // Takes item si from the global counter and publishes it; a
-            // valid item's Q tiles are prefetched into L2.
-            auto fetch = [&](int si) -> int {
-                const int slot = si & 3;
-                if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
-                                                 (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
-                    return -1;
-                const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
-                const int w = (long long)t < pair_items(p) ? (int)t : -1;
-                item_ring[slot] = w;
-                mbar_arrive(bar_ifull0 + 8 * slot);
-                if (w >= 0) {
-                    PairSeg nx;
-                    pair_item(p, w, nx);
-                    for (int x = 0; x < 2; ++x) {
-                        tma_prefetch_3d(&tm_q, 0, nx.qrow0, nx.qhead + x);
-                        tma_prefetch_3d(&tm_q, 64, nx.qrow0, nx.qhead + x);
-                    }
-                }
-                return w;
-            };
             int si = 0;
-            int w = fetch(0);
-            while (ok && w >= 0) {
-                pair_item(p, w, sg);
+            long long g = 0, kiss = 0;
+            while (ok && next_seg(si, true, ok)) {
                 // the Q buffer was last read by the QKs of item si - 1
                 if (si >= 1 && !(ok = mbar_wait(bar_qfree, (uint32_t)((si - 1) & 1), abort_flag)))
                     break;
@@ -236,9 +203,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                 bar_qfull);
                 }
                 ++si;
-                const int wn = fetch(si); // the next item, ahead of its turn
-                if (!ok)
-                    break;
                 for (int it = 0; it < sg.nt; ++it, ++g) {
                     const int s = (int)(g & 1);
                     // stage s was last read by QK_A and QK_B of tile g - 2
@@ -255,7 +219,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                 ks, sg.kvhead, bar_kfull(s));
                     kiss = g + 1;
                 }
-                w = wn;
             }
             // this CTA takes no more items; the last CTA resets the pair
             __threadfence();
@@ -280,7 +243,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             bool ok = true;
             int si = 0;
             long long g = 0, viss = 0;
-            while (ok && next_seg(si, ok)) {
+            while (ok && next_seg(si, false, ok)) {
                 ++si;
                 for (int it = 0; it < sg.nt; ++it, ++g) {
                     const int s = (int)(g & 1);
@@ -336,7 +299,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             auto wait_k = [&](long long jg) {
                 return mbar_wait(bar_kfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1), abort_flag);
             };
-            while (ok && next_seg(si, ok)) {
+            while (ok && next_seg(si, false, ok)) {
                 if (!(ok = mbar_wait(bar_qfull, (uint32_t)(si & 1), abort_flag)))
                     break;
                 if (!(ok = wait_k(j)))
@@ -391,95 +354,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
         }
     }
-    } else if (warp >= 12) {
-        // -------------------------------------------------------- epilogue
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPairRegsEpi));
-        const int wq = warp & 3;          // TMEM lane quarter
-        const int row = wq * 32 + lane;
-        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-        // Rows go out through this warp's 4 KB staging area, one 64-column
-        // half at a time, so that each global store writes four 128-byte row
-        // pieces instead of 16-byte pieces of 32 rows.  Chunk c (16 bytes)
-        // of row l sits at l * 128 + ((c ^ (l & 7)) << 4): conflict-free both
-        // for a lane writing its own row and for 8 lanes reading one row.
-        const uint32_t epi = base + kPairSmemEpi + (uint32_t)wq * (32 * 128);
-        bool ok = true;
-        long long j = 0;
-        int si = 0;
-        for (;;) {
-            const bool got = next_seg(si, ok);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!got || !ok)
-                break;
-            const long long jl = j + sg.nt - 1; // last PV of the item
-#pragma unroll 1
-            for (int x = 0; x < 2; ++x) {
-                ok = __all_sync(0xffffffffu,
-                                mbar_wait(bar_lfull(x), (uint32_t)(si & 1), abort_flag) &&
-                                    mbar_wait(bar_odone(x, (int)(jl & 1)),
-                                              (uint32_t)((jl >> 1) & 1), abort_flag));
-                if (!ok)
-                    break;
-                tc_fence_after();
-                const float *lmx = lm + (((si & 1) * 2 + x) * 2) * 128;
-                const float l = lmx[row], m_used = lmx[128 + row];
-                const float inv = (l > 0.f) ? 1.f / l : 0.f;
-                const float lse_v = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-                const uint32_t t_o = tmem + 256 + (uint32_t)x * 128;
-                const size_t head_row0 = (size_t)(sg.qhead + x) * 2 * p.L + sg.qrow0;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        const int q4 = 2 * h + q;
-                        uint32_t o[32];
-                        tmem_ld32(t_o + lane_off + q4 * 32, o);
-                        tmem_wait_ld();
-                        if (q4 == kTcD / 32 - 1) {
-                            // O_x fully read: the next item's first PV_x may go
-                            tc_fence_before();
-                            mbar_arrive(bar_ofree(x));
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            const uint32_t c = (uint32_t)(q * 4 + i / 8);
-                            const uint32_t a = epi + (uint32_t)lane * 128 +
-                                               ((c ^ (uint32_t)(lane & 7)) << 4);
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a),
-                                         "r"(pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv)),
-                                         "r"(pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv)),
-                                         "r"(pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv)),
-                                         "r"(pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv))
-                                         : "memory");
-                        }
-                    }
-                    __syncwarp();
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int r = 4 * i + (lane >> 3); // row within the warp's 32
-                        const uint32_t cc = (uint32_t)(lane & 7);
-                        uint32_t x0, x1, x2, x3;
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                                     : "r"(epi + (uint32_t)r * 128 + ((cc ^ (uint32_t)(r & 7)) << 4))
-                                     : "memory");
-                        const int trow = wq * 32 + r;
-                        if (trow < sg.nrows)
-                            reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * kTcD)[h * 8 + cc] =
-                                make_uint4(x0, x1, x2, x3);
-                    }
-                    __syncwarp();
-                }
-                if (row < sg.nrows)
-                    p.lse[head_row0 + row] = lse_v;
-            }
-            if (!ok)
-                break;
-            j += sg.nt;
-            ++si;
-        }
     } else {
-        // ------------------------------------------------------ softmax
+        // -------------------------------------------- softmax + epilogue
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPairRegsSoftmax));
         const int x = warp >> 2;          // 0: tile A, 1: tile B
         const int wq = warp & 3;          // TMEM lane quarter
@@ -492,7 +368,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         long long j = 0;
         int si = 0;
         for (;;) {
-            const bool got = next_seg(si, ok);
+            const bool got = next_seg(si, false, ok);
             ok = __all_sync(0xffffffffu, ok);
             if (!got || !ok)
                 break;
@@ -512,8 +388,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     break;
                 tc_fence_after();
                 const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
-                const long long jp = jg - 1; // PV_x(jp) done => O_x stable
-                ok = softmax_tile<kEmuExp2>(
+                const long long jp = jg - 1;
+                ok = softmax_tile<kEmuExp2, false>(
                     t_s + lane_off, t_o + lane_off, full, sp, ks, khi, sl2, jj >= 1, m_used, l,
                     [&] {
                         return mbar_wait(bar_odone(x, (int)(jp & 1)), (uint32_t)((jp >> 1) & 1),
@@ -527,11 +403,65 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             }
             if (!ok)
                 break;
-            // hand the row's sum and maximum to the epilogue warpgroup
-            float *lmx = lm + (((si & 1) * 2 + x) * 2) * 128;
-            lmx[row] = l;
-            lmx[128 + row] = m_used;
-            mbar_arrive(bar_lfull(x));
+            {
+                const long long jl = j + sg.nt - 1; // last PV of the item
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_odone(x, (int)(jl & 1)),
+                                                       (uint32_t)((jl >> 1) & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+            }
+            // ------------------------------------------------ epilogue
+            // Rows go out through this warp's 4 KB staging area, one
+            // 64-column half at a time, so that each global store writes four
+            // 128-byte row pieces instead of 16-byte pieces of 32 rows.  Chunk
+            // c (16 bytes) of row l sits at l * 128 + ((c ^ (l & 7)) << 4).
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            const float lse_v = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+            const size_t head_row0 = (size_t)(sg.qhead + x) * 2 * p.L + sg.qrow0;
+            const uint32_t epi = base + kPairSmemEpi + (uint32_t)warp * (32 * 128);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int q4 = 2 * h + q;
+                    uint32_t o[32];
+                    tmem_ld32(t_o + lane_off + q4 * 32, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        const uint32_t cch = (uint32_t)(q * 4 + i / 8);
+                        const uint32_t a = epi + (uint32_t)lane * 128 +
+                                           ((cch ^ (uint32_t)(lane & 7)) << 4);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv)),
+                                     "r"(pack_bf16x2(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv))
+                                     : "memory");
+                    }
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int r = 4 * i + (lane >> 3); // row within the warp's 32
+                    const uint32_t cc = (uint32_t)(lane & 7);
+                    uint32_t x0, x1, x2, x3;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                                 : "r"(epi + (uint32_t)r * 128 + ((cc ^ (uint32_t)(r & 7)) << 4))
+                                 : "memory");
+                    const int trow = wq * 32 + r;
+                    if (trow < sg.nrows)
+                        reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * kTcD)[h * 8 + cc] =
+                            make_uint4(x0, x1, x2, x3);
+                }
+                __syncwarp();
+            }
+            if (row < sg.nrows)
+                p.lse[head_row0 + row] = lse_v;
+            tc_fence_before();
+            mbar_arrive(bar_ofree(x));
             j += sg.nt;
             ++si;
         }

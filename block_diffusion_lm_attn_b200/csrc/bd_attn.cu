@@ -56,8 +56,7 @@ bool pair_kernel_usable()
         cudaFuncAttributes a;
         u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel) == cudaSuccess &&
              (long long)a.numRegs * bd::kPairThreads >=
-                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther +
-                     128LL * bd::kPairRegsEpi)
+                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther)
                 ? 1
                 : 0;
         usable.store(u);
@@ -664,17 +663,23 @@ bd_status bd_sprint_prune(const void *k_cache, const void *v_cache,
     double *sc = score ? score
                        : reinterpret_cast<double *>(static_cast<char *>(workspace) +
                                                     round256((size_t)B * S_cap * sizeof(double)));
-    dim3 gn((S_cap + 7) / 8, B);
+    dim3 gn((S_cap + 8 * bd::kNormPos - 1) / (8 * bd::kNormPos), B);
     bd::bd_sprint_norm_kernel<<<gn, 256, 0, stream>>>(static_cast<const bf16 *>(k_cache),
                                                       cache_len, norm, Hkv, d, S_cap);
     if (cudaGetLastError() != cudaSuccess)
         return BD_ERR_CUDA;
-    bd::bd_sprint_select_kernel<<<B, bd::kSelThreads, 0, stream>>>(
-        norm, cache_len, conf, modality, (double)alpha, (double)keep_text, (double)keep_image,
-        sc, kept, new_len, S_cap);
+    // a thread's run of the prefix fits its registers up to 16 positions
+    if (S_cap <= 16 * bd::kSelThreads)
+        bd::bd_sprint_select_kernel<16><<<B, bd::kSelThreads, 0, stream>>>(
+            norm, cache_len, conf, modality, (double)alpha, (double)keep_text,
+            (double)keep_image, sc, kept, new_len, S_cap);
+    else
+        bd::bd_sprint_select_kernel<0><<<B, bd::kSelThreads, 0, stream>>>(
+            norm, cache_len, conf, modality, (double)alpha, (double)keep_text,
+            (double)keep_image, sc, kept, new_len, S_cap);
     if (cudaGetLastError() != cudaSuccess)
         return BD_ERR_CUDA;
-    bd::bd_sprint_compact_kernel<<<gn, 256, 0, stream>>>(
+    bd::bd_sprint_compact_kernel<<<dim3((S_cap + 7) / 8, B), 256, 0, stream>>>(
         static_cast<const bf16 *>(k_cache), static_cast<const bf16 *>(v_cache), kept, new_len,
         static_cast<bf16 *>(k_out), static_cast<bf16 *>(v_out), Hkv, d, S_cap);
     return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;

@@ -104,39 +104,61 @@ __global__ void __launch_bounds__(256)
 // sparse prefix retention
 
 // |k_p|_2 over all kv-heads and dims of position p, for p < cache_len[i]:
-// norm[i][p] in fp64.  One warp per position; lane l reads 16-byte pieces
-// of the position's Hkv rows (two rows per warp load, each row contiguous).
+// norm[i][p] in fp64.  A warp takes kNormPos consecutive positions, lane l
+// reading 16-byte pieces of their Hkv rows (each row contiguous, two rows per
+// warp load); all of a warp's loads are issued before the sums.
+constexpr int kNormPos = 4;
+
 __global__ void __launch_bounds__(256)
     bd_sprint_norm_kernel(const bf16 *k_cache, const int32_t *cache_len,
                           double *norm, int Hkv, int d, int S_cap)
 {
     const int i = blockIdx.y;
-    const int p = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int pbase = (blockIdx.x * 8 + (threadIdx.x >> 5)) * kNormPos;
     const int lane = threadIdx.x & 31;
     const int len = cache_len[i];
-    if (p >= S_cap || p >= len || len > S_cap)
+    if (pbase >= len || len > S_cap)
         return;
     const int vec_per_row = d / 8;
-    const int nvec = Hkv * vec_per_row;
-    double ss = 0.0;
-    for (int e = lane; e < nvec; e += 32) {
-        const int h = e / vec_per_row, c = e % vec_per_row;
-        const uint4 x = *reinterpret_cast<const uint4 *>(
-            k_cache + (((size_t)i * Hkv + h) * S_cap + p) * d + (size_t)c * 8);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    const int nvec = Hkv * vec_per_row; // multiple of 4 (d >= 32)
+    double ss[kNormPos];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            const double lo = (double)__uint_as_float(w[t] << 16);
-            const double hi = (double)__uint_as_float(w[t] & 0xffff0000u);
-            ss = fma(lo, lo, ss);
-            ss = fma(hi, hi, ss);
+    for (int q = 0; q < kNormPos; ++q)
+        ss[q] = 0.0;
+    for (int e0 = 0; e0 < nvec; e0 += 32) {
+        const int e = e0 + lane;
+        uint4 x[kNormPos];
+#pragma unroll
+        for (int q = 0; q < kNormPos; ++q) {
+            const int p = pbase + q;
+            x[q] = make_uint4(0, 0, 0, 0);
+            if (e < nvec && p < len) {
+                const int h = e / vec_per_row, c = e % vec_per_row;
+                x[q] = *reinterpret_cast<const uint4 *>(
+                    k_cache + (((size_t)i * Hkv + h) * S_cap + p) * d + (size_t)c * 8);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < kNormPos; ++q) {
+            const uint32_t w[4] = {x[q].x, x[q].y, x[q].z, x[q].w};
+#pragma unroll
+            for (int t4 = 0; t4 < 4; ++t4) {
+                // bf16 squares are exact in fp64
+                const double lo = (double)__uint_as_float(w[t4] << 16);
+                const double hi = (double)__uint_as_float(w[t4] & 0xffff0000u);
+                ss[q] = fma(lo, lo, ss[q]);
+                ss[q] = fma(hi, hi, ss[q]);
+            }
         }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0)
-        norm[(size_t)i * S_cap + p] = sqrt(ss);
+    for (int q = 0; q < kNormPos; ++q) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            ss[q] += __shfl_xor_sync(0xffffffffu, ss[q], o);
+        if (lane == 0 && pbase + q < len)
+            norm[(size_t)i * S_cap + pbase + q] = sqrt(ss[q]);
+    }
 }
 
 constexpr int kSelThreads = 1024;
@@ -197,7 +219,10 @@ __device__ int block_scan_excl(int v, int *red, int &total)
 //   kept[i][0 .. new_len-1] = kept positions in increasing order, then -1.
 // The threshold of each modality is found by an 8-pass radix select (8 bits
 // per pass) over the score keys; positions are visited in contiguous
-// per-thread runs so that the final scan keeps position order.
+// per-thread runs so that the final scan keeps position order.  With
+// PER > 0 a thread's run (at most PER positions) is held in registers;
+// PER = 0 reads it from memory on every pass (long prefixes).
+template <int PER>
 __global__ void __launch_bounds__(kSelThreads)
     bd_sprint_select_kernel(const double *norm, const int32_t *cache_len,
                             const float *conf, const uint8_t *modality,
@@ -226,34 +251,51 @@ __global__ void __launch_bounds__(kSelThreads)
     // this thread's contiguous run of positions [p0, p1)
     const int per = (len + blockDim.x - 1) / blockDim.x;
     const int p0 = min(len, tid * per), p1 = min(len, p0 + per);
+    const int cnt = p1 - p0;
 
     double part = 0.0;
     for (int p = p0; p < p1; ++p)
         part += norm[row + p];
     const double mean = block_sum(part, red_d) / (double)max(len, 1);
-    for (int p = p0; p < p1; ++p) {
+    // run cache: score key and modality bit of each position of the run;
+    // every loop over the run is unrolled to RMAX with an early exit, so
+    // the cache stays in registers
+    constexpr int RMAX = PER > 0 ? PER : 64;
+    constexpr int R = PER > 0 ? PER : 1;
+    unsigned long long rk[R];
+    uint64_t rm = 0;
+    int nimg = 0;
+#pragma unroll
+    for (int u = 0; u < RMAX; ++u) {
+        if (u >= cnt)
+            break;
+        const int p = p0 + u;
         // separate roundings, no fused multiply-add: the same arithmetic as
         // the plain definition, so equal inputs give equal scores
         const double inorm = mean > 0.0 ? __ddiv_rn(norm[row + p], mean) : 0.0;
-        score[row + p] = __dadd_rn(__dmul_rn(alpha, inorm),
-                                   __dmul_rn(__dadd_rn(1.0, -alpha), (double)conf[row + p]));
-    }
-    __syncthreads();
-
-    // kept flags live in the kept row itself until the final compaction:
-    // 1 = kept, 0 = dropped.  Both modalities are selected together: an
-    // 8-pass radix select (8 bits per pass) of each modality's want-th
-    // largest score key, one 256-bin histogram per modality.
-    {
-        int cnt1 = 0, cnt = 0;
-        for (int p = p0; p < p1; ++p) {
-            cnt1 += modality[row + p] != 0;
-            ++cnt;
+        const double sc = __dadd_rn(__dmul_rn(alpha, inorm),
+                                    __dmul_rn(__dadd_rn(1.0, -alpha), (double)conf[row + p]));
+        score[row + p] = sc;
+        const int m = modality[row + p] != 0;
+        nimg += m;
+        if (PER > 0) {
+            rk[PER > 0 ? u : 0] = dkey(sc);
+            rm |= (uint64_t)m << u;
         }
-        const int n_img = block_sum(cnt1, red_i);
-        const int n_all = block_sum(cnt, red_i);
+    }
+    // key and modality of run position u
+    auto key_at = [&](int u, int &m) -> unsigned long long {
+        if (PER > 0) {
+            m = (int)((rm >> u) & 1u);
+            return rk[PER > 0 ? u : 0];
+        }
+        m = modality[row + p0 + u] != 0;
+        return dkey(score[row + p0 + u]);
+    };
+    {
+        const int n_img = block_sum(nimg, red_i);
         if (tid == 0) {
-            const int n_m[2] = {n_all - n_img, n_img};
+            const int n_m[2] = {len - n_img, n_img};
             for (int m = 0; m < 2; ++m) {
                 const double r = m == 0 ? keep_text : keep_image;
                 long long want = (long long)floor(r * (double)n_m[m] + 0.5);
@@ -265,6 +307,9 @@ __global__ void __launch_bounds__(kSelThreads)
         }
         __syncthreads();
     }
+    // kept flags live in the kept row itself until the final compaction:
+    // 1 = kept, 0 = dropped.  Both modalities are selected together, one
+    // 256-bin histogram per modality.
     for (int pass = 0; pass < 8; ++pass) {
         const int shift = 56 - 8 * pass;
         for (int k = tid; k < 512; k += blockDim.x)
@@ -272,9 +317,12 @@ __global__ void __launch_bounds__(kSelThreads)
         __syncthreads();
         const unsigned long long hmask = pass == 0 ? 0ull : (~0ull << (shift + 8));
         const unsigned long long pre0 = s_prefix[0], pre1 = s_prefix[1];
-        for (int p = p0; p < p1; ++p) {
-            const int m = modality[row + p] != 0;
-            const unsigned long long key = dkey(score[row + p]);
+#pragma unroll
+        for (int u = 0; u < RMAX; ++u) {
+            if (u >= cnt)
+                break;
+            int m;
+            const unsigned long long key = key_at(u, m);
             if ((key & hmask) == (m ? pre1 : pre0))
                 atomicAdd(&hist[m * 256 + ((key >> shift) & 255)], 1u);
         }
@@ -314,53 +362,60 @@ __global__ void __launch_bounds__(kSelThreads)
         }
         __syncthreads();
     }
-    for (int m = 0; m < 2; ++m) {
-        // keys above the threshold are kept; of the keys equal to it, the
-        // s_need lowest positions
-        const bool any = s_want[m] > 0;
-        const unsigned long long thr = s_prefix[m];
-        const int need_eq = any ? s_need[m] : 0;
-        int eq = 0;
-        for (int p = p0; p < p1; ++p)
-            if ((modality[row + p] != 0) == m && any && dkey(score[row + p]) == thr)
-                ++eq;
-        int tot_eq;
-        int before = block_scan_excl(eq, red_i, tot_eq);
-        for (int p = p0; p < p1; ++p) {
-            if ((modality[row + p] != 0) != m)
-                continue;
-            int keep = 0;
-            if (any) {
-                const unsigned long long key = dkey(score[row + p]);
-                if (key > thr)
-                    keep = 1;
-                else if (key == thr)
-                    keep = (before++ < need_eq);
-            }
-            kept[row + p] = keep;
+    // keys above a modality's threshold are kept; of the keys equal to it,
+    // its s_need lowest positions
+    const unsigned long long thr0 = s_prefix[0], thr1 = s_prefix[1];
+    const bool any0 = s_want[0] > 0, any1 = s_want[1] > 0;
+    int eq[2] = {0, 0};
+#pragma unroll
+    for (int u = 0; u < RMAX; ++u) {
+        if (u >= cnt)
+            break;
+        int m;
+        const unsigned long long key = key_at(u, m);
+        eq[m] += (m ? any1 : any0) && key == (m ? thr1 : thr0);
+    }
+    int tot0, tot1;
+    int before0 = block_scan_excl(eq[0], red_i, tot0);
+    int before1 = block_scan_excl(eq[1], red_i, tot1);
+    const int need0 = any0 ? s_need[0] : 0, need1 = any1 ? s_need[1] : 0;
+    int mine = 0;
+    uint64_t keepbits = 0;
+#pragma unroll
+    for (int u = 0; u < RMAX; ++u) {
+        if (u >= cnt)
+            break;
+        int m;
+        const unsigned long long key = key_at(u, m);
+        const unsigned long long thr = m ? thr1 : thr0;
+        int keep = 0;
+        if (m ? any1 : any0) {
+            if (key > thr)
+                keep = 1;
+            else if (key == thr)
+                keep = m ? (before1++ < need1) : (before0++ < need0);
         }
-        __syncthreads();
+        if (PER > 0)
+            keepbits |= (uint64_t)keep << u;
+        else
+            kept[row + p0 + u] = keep;
+        mine += keep;
     }
 
     // stable compaction of the kept positions
-    int mine = 0;
-    for (int p = p0; p < p1; ++p)
-        mine += kept[row + p];
     int total;
     int dst = block_scan_excl(mine, red_i, total);
-    // read the flags of this thread's run before any thread overwrites them
-    // with positions: a thread's destinations can reach into the runs of
-    // threads before it only, whose flags those threads already hold
-    int flags[64];
-    int nf = 0;
-    for (int p = p0; p < p1 && nf < 64; ++p)
-        flags[nf++] = kept[row + p];
-    __syncthreads();
-    if (per <= 64) {
-        for (int p = p0, k = 0; p < p1; ++p, ++k)
-            if (flags[k])
-                kept[row + dst++] = p;
+    if (PER == 0) {
+        // the flags of this thread's run are in memory: read them before
+        // any thread overwrites them with positions (a thread's
+        // destinations reach into the runs of threads before it only)
+        for (int u = 0; u < cnt; ++u)
+            keepbits |= (uint64_t)kept[row + p0 + u] << u;
+        __syncthreads();
     }
+    for (int u = 0; u < cnt; ++u)
+        if ((keepbits >> u) & 1u)
+            kept[row + dst++] = p0 + u;
     __syncthreads();
     for (int p = total + tid; p < S_cap; p += blockDim.x)
         kept[row + p] = -1;

@@ -144,6 +144,14 @@ def test_sprint_ragged_lengths(d):
     check_sprint(k, v, conf, mod, cl, 0.5, 1.0, 0.8)
 
 
+def test_sprint_prefix_longer_than_register_runs():
+    """Prefixes over 16 x 1024 positions take the selection path that keeps
+    each thread's run in memory."""
+    lens = [20000, 16385, 300]
+    k, v, conf, mod, cl = sprint_inputs(3, 1, 32, 20100, lens, 76)
+    check_sprint(k, v, conf, mod, cl, 0.5, 0.6, 0.8)
+
+
 def test_sprint_full_size_denoise_cache():
     """The denoising-decode cache (B=16, Hkv=8, d=128, 8192 cached tokens):
     3/4 image tokens then text, as a prompt of an image and a question."""
