@@ -157,11 +157,15 @@ constexpr int kKvSmemBytes = kKvSmemBar + 512 + 1024;
 static_assert(kKvStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(kKvSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
-constexpr int kBwdThreads = 192; // 4 compute warps, producer, MMA issuer
+// 8 compute warps (two per TMEM lane quarter, each taking half of a row's
+// columns), a producer warp and an MMA warp
+constexpr int kBwdThreads = 320;
+constexpr int kBwdProducerWarp = 8, kBwdMmaWarp = 9;
 
-// Roles: warps 0-3 compute P^T and dS^T (thread t = key row t = TMEM lane
-// t) and write dK, dV out; warp 4 loads (TMA for tiles, plain loads for the
-// per-row lse2 and D) and fetches work items; warp 5 issues the MMAs.
+// Roles: warps 0-7 compute P^T and dS^T (warp w: key rows of TMEM lane
+// quarter w & 3, half w >> 2 of each step's query columns) and write dK, dV
+// out; warp 8 loads (TMA for tiles, plain loads for the per-row lse2 and D)
+// and fetches work items; warp 9 issues the MMAs.
 // TMEM: dV [0,128), dK [128,256); two buffers x of S^T [256 + 128x, +64)
 // and dP^T [320 + 128x, +64); P^T (bf16) overwrites its S^T, dS^T its dP^T.
 // Per step s (64 query rows, buffer x = s & 1):
@@ -208,20 +212,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(bar_sfull(x), 1);
-            mbar_init(bar_pfull(x), 4); // one arrival per compute warp
+            mbar_init(bar_pfull(x), 8); // one arrival per compute warp
         }
         mbar_init(bar_odone, 1);
-        mbar_init(bar_ofree, 128);
+        mbar_init(bar_ofree, 8);
         mbar_init(bar_final, 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_ifull0 + 8 * i, 1);
-            mbar_init(bar_iempty0 + 8 * i, 129); // MMA + 128 compute threads
+            mbar_init(bar_iempty0 + 8 * i, 257); // MMA + 256 compute threads
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32((const void *)tmem_slot)), "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -258,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return true;
     };
 
-    if (warp == 4) {
+    if (warp == kBwdProducerWarp) {
         // ------------------------------------------------------ producer
         bool ok = true;
         int si = 0;
@@ -345,7 +349,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (long long x = iss > kKvStages ? iss - kKvStages : 0; x < iss; ++x)
                 drain(bar_full((int)(x % kKvStages)), (uint32_t)((x / kKvStages) & 1));
         }
-    } else if (warp == 5) {
+    } else if (warp == kBwdMmaWarp) {
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(kTcM, kBwdSub, 0);  // S^T, dP^T
@@ -376,15 +380,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             auto issue_grad = [&](long long gg, bool first) {
                 const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
                 const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
+                // K-step kk covers queries 16 kk .. 16 kk + 15, packed by the
+                // compute warps of half kk / 2 at columns 32 (kk / 2) + 8 (kk % 2)
 #pragma unroll
                 for (int kk = 0; kk < kBwdSub / 16; ++kk) {
+                    const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bdo = smem_desc_sw128(sb + kSubBytes + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts(t_dv, t_st(x) + kk * 8, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(t_dv, t_st(x) + acol, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kBwdSub / 16; ++kk) {
+                    const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bq = smem_desc_sw128(sb + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts(t_dk, t_dp(x) + kk * 8, bq, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts(t_dk, t_dp(x) + acol, bq, idesc_g, (!first || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(bar_empty(st));
             };
@@ -426,8 +434,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else {
         // ------------------------------------------ P^T, dS^T and epilogue
-        const int row = threadIdx.x; // key row of the tile = TMEM lane
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // warp w: key rows 32 (w & 3) .. +31 (TMEM lane quarter), query
+        // columns 32 hc .. 32 hc + 31 of each 64-row step, hc = w >> 2.  The
+        // packed P^T / dS^T of half hc go to columns 32 hc .. 32 hc + 15 of
+        // the S^T / dP^T buffer: inside the columns this warp itself read,
+        // so the other half's loads are never overwritten.
+        const int wq = warp & 3, hc = warp >> 2;
+        const int row = wq * 32 + lane; // key row of the tile = TMEM lane
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
         long long g = 0;
@@ -455,31 +469,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!ok)
                     break;
                 tc_fence_after();
-                uint32_t sr[64], dr[64];
-                tmem_ld32(t_st(x) + lane_off, sr);
-                tmem_ld32(t_st(x) + lane_off + 32, sr + 32);
-                tmem_ld32(t_dp(x) + lane_off, dr);
-                tmem_ld32(t_dp(x) + lane_off + 32, dr + 32);
+                uint32_t sr[32], dr[32];
+                tmem_ld32(t_st(x) + lane_off + 32 * hc, sr);
+                tmem_ld32(t_dp(x) + lane_off + 32 * hc, dr);
                 tmem_wait_ld();
                 const float *sl = reinterpret_cast<const float *>(
-                    sbase + kKvSmemRows + st * kKvRowsBytes);
+                                      sbase + kKvSmemRows + st * kKvRowsBytes) + 32 * hc;
                 const int hi = rg == 0 ? it.hi0 : it.hi1;
                 const int flo = rg == 0 ? it.flo0 : it.flo1;
                 const int fhi = rg == 0 ? it.fhi0 : it.fhi1;
                 const bool full = qs >= flo && qs + kBwdSub <= fhi && qs + kBwdSub <= hi;
-                uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
+                uint32_t mw = 0xffffffffu;
                 if (!full) {
+                    const int q0 = qs + 32 * hc;
                     const int e = min(hi, qs + kBwdSub);
-                    const int lo0 = max(ksp.a0, qs) - qs, hi0 = min(ksp.a1, e) - qs;
-                    const int lo1 = max(ksp.a2, qs) - qs, hi1 = min(ksp.a3, e) - qs;
-#pragma unroll
-                    for (int w = 0; w < 2; ++w)
-                        mw[w] = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
-                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
+                    const int lo0 = max(ksp.a0, q0) - q0, hi0 = min(ksp.a1, e) - q0;
+                    const int lo1 = max(ksp.a2, q0) - q0, hi1 = min(ksp.a3, e) - q0;
+                    mw = range_bits(lo0, hi0) | range_bits(lo1, hi1);
                 }
-                uint32_t pk[32], dk[32];
+                uint32_t pk[16], dk[16];
 #pragma unroll
-                for (int c = 0; c < kBwdSub; c += 4) {
+                for (int c = 0; c < 32; c += 4) {
                     const float4 l4 = *reinterpret_cast<const float4 *>(sl + c);
                     const float4 d4 = *reinterpret_cast<const float4 *>(sl + kBwdSub + c);
                     const float la[4] = {l4.x, l4.y, l4.z, l4.w};
@@ -489,7 +499,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int u = 0; u < 4; ++u) {
                         const int cc = c + u;
                         float xx = fmaf(__uint_as_float(sr[cc]), sl2, -la[u]);
-                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u))
+                        if (!((mw >> cc) & 1u))
                             xx = -INFINITY;
                         pv[u] = ex2(xx);
                         dv[u] = pv[u] * (__uint_as_float(dr[cc]) - da[u]);
@@ -499,10 +509,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
                     dk[c / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
                 }
-                tmem_st16(t_st(x) + lane_off, pk);
-                tmem_st16(t_st(x) + lane_off + 16, pk + 16);
-                tmem_st16(t_dp(x) + lane_off, dk);
-                tmem_st16(t_dp(x) + lane_off + 16, dk + 16);
+                tmem_st16(t_st(x) + lane_off + 32 * hc, pk);
+                tmem_st16(t_dp(x) + lane_off + 32 * hc, dk);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -515,16 +523,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            // epilogue: dV and scale * dK, bf16, one row per thread
+            // epilogue: dV and scale * dK, bf16; this thread's row, columns
+            // 64 hc .. 64 hc + 63
             const bool valid = row < it.nkeys;
             const size_t grow = (size_t)it.kvhead * 2 * p.L + it.krow0 + row;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
-                const uint32_t tb = (which == 0 ? t_dv : t_dk) + lane_off;
+                const uint32_t tb = (which == 0 ? t_dv : t_dk) + lane_off + 64 * hc;
                 const float mul = which == 0 ? 1.f : p.scale;
-                bf16 *dst = (which == 0 ? p.dv : p.dk) + grow * kTcD;
+                bf16 *dst = (which == 0 ? p.dv : p.dk) + grow * kTcD + 64 * hc;
 #pragma unroll
-                for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                for (int q4 = 0; q4 < 2; ++q4) {
                     uint32_t o[32];
                     tmem_ld32(tb + q4 * 32, o);
                     tmem_wait_ld();
@@ -542,7 +551,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(bar_ofree);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_ofree);
             g += it.nt;
             ++si;
         }
@@ -550,7 +561,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
@@ -566,8 +577,9 @@ constexpr int kDqSmemBar = kDqSmemRing + 2 * 2 * kTileBytes;
 constexpr int kDqSmemBytes = kDqSmemBar + 512 + 1024;
 static_assert(kDqSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
-// Roles: warps 0-3 compute dS (thread t = query row t) and write dQ out;
-// warp 4 loads and fetches items; warp 5 issues the MMAs.  TMEM: S [0,128),
+// Roles: warps 0-7 compute dS (warp w: query rows of TMEM lane quarter
+// w & 3, half w >> 2 of the key columns) and write dQ out; warp 8 loads and
+// fetches items; warp 9 issues the MMAs.  TMEM: S [0,128),
 // dP [128,256), dQ [256,384), two dS buffers (bf16) [384,448), [448,512).
 // Per key tile j: S = Q K^T and dP = dO V^T (after the compute warps have
 // read S, dP of tile j - 1 into registers), then dQ += dS(j - 1) K(j - 1).
@@ -592,7 +604,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar_dsfull = [&](int x) { return bar0 + 64 + 8 * x; };
     auto bar_dsfree = [&](int x) { return bar0 + 80 + 8 * x; };
     const uint32_t bar_qdone = bar0 + 96;  // the item's last dQ retired
-    const uint32_t bar_dqfree = bar0 + 104; // dQ read out (128)
+    const uint32_t bar_dqfree = bar0 + 104; // dQ read out
     const uint32_t bar_final = bar0 + 112;
     const uint32_t bar_ifull0 = bar0 + 120;
     const uint32_t bar_iempty0 = bar0 + 152;
@@ -608,23 +620,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar_kvfull(s), 1);
             mbar_init(bar_kvempty(s), 1);
-            mbar_init(bar_dsfull(s), 4); // one arrival per compute warp
+            mbar_init(bar_dsfull(s), 8); // one arrival per compute warp
             mbar_init(bar_dsfree(s), 1);
         }
         mbar_init(bar_sfull, 1);
-        mbar_init(bar_sfree, 4);
+        mbar_init(bar_sfree, 8);
         mbar_init(bar_qdone, 1);
-        mbar_init(bar_dqfree, 128);
+        mbar_init(bar_dqfree, 8);
         mbar_init(bar_final, 1);
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar_ifull0 + 8 * i, 1);
-            mbar_init(bar_iempty0 + 8 * i, 129);
+            mbar_init(bar_iempty0 + 8 * i, 257); // MMA + 256 compute threads
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32((const void *)tmem_slot)), "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -667,7 +679,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         return t < sg.n0 ? sg.lo0 + t * kTcN : sg.lo1 + (t - sg.n0) * kTcN;
     };
 
-    if (warp == 4) {
+    if (warp == kBwdProducerWarp) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             bool ok = true;
@@ -714,7 +726,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (long long x = iss > 2 ? iss - 2 : 0; x < iss; ++x)
                 drain(bar_kvfull((int)(x & 1)), (uint32_t)((x >> 1) & 1));
         }
-    } else if (warp == 5) {
+    } else if (warp == kBwdMmaWarp) {
         // ---------------------------------------------------- MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(kTcM, kTcN, 0);
@@ -792,8 +804,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else {
         // ---------------------------------------------- dS and epilogue
-        const int row = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // warp w: query rows of TMEM lane quarter w & 3, key columns
+        // 64 hc .. 64 hc + 63 of each tile (hc = w >> 2); dS is elementwise,
+        // so the two halves of a row need nothing from each other.
+        const int wq = warp & 3, hc = warp >> 2;
+        const int row = wq * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
         const float sl2 = p.scale_log2;
         bool ok = true;
         long long j = 0;
@@ -822,15 +838,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     break;
                 tc_fence_after();
                 const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
-                uint32_t mw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+                uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
                 if (!full) {
+                    const int k0 = ks + 64 * hc;
                     const int e = min(khi, ks + kTcN);
-                    const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
-                    const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
+                    const int lo0 = max(sp.a0, k0) - k0, hi0 = min(sp.a1, e) - k0;
+                    const int lo1 = max(sp.a2, k0) - k0, hi1 = min(sp.a3, e) - k0;
 #pragma unroll
-                    for (int w = 0; w < 4; ++w)
+                    for (int w = 0; w < 2; ++w)
                         mw[w] = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
                                 range_bits(lo1 - 32 * w, hi1 - 32 * w);
+                }
+                uint32_t sr[64], dr[64], pk[32];
+                tmem_ld32(t_s + lane_off + 64 * hc, sr);
+                tmem_ld32(t_s + lane_off + 64 * hc + 32, sr + 32);
+                tmem_ld32(t_dp + lane_off + 64 * hc, dr);
+                tmem_ld32(t_dp + lane_off + 64 * hc + 32, dr + 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_sfree); // S, dP may be overwritten
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    float x0 = fmaf(__uint_as_float(sr[c]), sl2, -lse2);
+                    float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2);
+                    if (!((mw[c >> 5] >> (c & 31)) & 1u))
+                        x0 = -INFINITY;
+                    if (!((mw[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u))
+                        x1 = -INFINITY;
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    pk[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[c]) - Dr),
+                                            p1 * (__uint_as_float(dr[c + 1]) - Dr));
                 }
                 // dS buffer x was last read by dQ of tile jg - 2 (issued
                 // while this warp worked on tile jg - 1)
@@ -841,36 +880,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         break;
                     tc_fence_after();
                 }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t sr[64], dr[64], pk[32];
-                    tmem_ld32(t_s + lane_off + 64 * h, sr);
-                    tmem_ld32(t_s + lane_off + 64 * h + 32, sr + 32);
-                    tmem_ld32(t_dp + lane_off + 64 * h, dr);
-                    tmem_ld32(t_dp + lane_off + 64 * h + 32, dr + 32);
-                    tmem_wait_ld();
-                    if (h == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive(bar_sfree); // S, dP may be overwritten
-                    }
-#pragma unroll
-                    for (int c = 0; c < 64; c += 2) {
-                        const int cc = 64 * h + c;
-                        float x0 = fmaf(__uint_as_float(sr[c]), sl2, -lse2);
-                        float x1 = fmaf(__uint_as_float(sr[c + 1]), sl2, -lse2);
-                        if (!((mw[cc >> 5] >> (cc & 31)) & 1u))
-                            x0 = -INFINITY;
-                        if (!((mw[(cc + 1) >> 5] >> ((cc + 1) & 31)) & 1u))
-                            x1 = -INFINITY;
-                        const float p0 = ex2(x0), p1 = ex2(x1);
-                        pk[c / 2] = pack_bf16x2(p0 * (__uint_as_float(dr[c]) - Dr),
-                                                p1 * (__uint_as_float(dr[c + 1]) - Dr));
-                    }
-                    tmem_st16(t_ds(x) + lane_off + 32 * h, pk);
-                    tmem_st16(t_ds(x) + lane_off + 32 * h + 16, pk + 16);
-                }
+                tmem_st16(t_ds(x) + lane_off + 32 * hc, pk);
+                tmem_st16(t_ds(x) + lane_off + 32 * hc + 16, pk + 16);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -883,10 +894,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok)
                 break;
             tc_fence_after();
+            // this thread's row, dQ columns 64 hc .. 64 hc + 63
 #pragma unroll
-            for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+            for (int q4 = 0; q4 < 2; ++q4) {
                 uint32_t o[32];
-                tmem_ld32(t_dq + lane_off + q4 * 32, o);
+                tmem_ld32(t_dq + lane_off + 64 * hc + q4 * 32, o);
                 tmem_wait_ld();
                 if (valid) {
                     const float mul = p.scale;
@@ -897,12 +909,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * mul, __uint_as_float(o[i + 3]) * mul);
                         v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * mul, __uint_as_float(o[i + 5]) * mul);
                         v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * mul, __uint_as_float(o[i + 7]) * mul);
-                        reinterpret_cast<uint4 *>(p.dq + grow * kTcD)[q4 * 4 + i / 8] = v4;
+                        reinterpret_cast<uint4 *>(p.dq + grow * kTcD + 64 * hc)[q4 * 4 + i / 8] = v4;
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(bar_dqfree);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_dqfree);
             j += sg.nt;
             ++si;
         }
@@ -910,7 +924,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kBwdMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
