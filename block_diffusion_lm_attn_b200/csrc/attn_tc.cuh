@@ -144,6 +144,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
     }
 }
 
+// mbar_wait by every lane of a converged warp; the result is the same in all
+// lanes (false if any lane's wait gave up)
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int *abort_flag)
+{
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
 __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *tm,
                                             int c0, int c1, int c2,
                                             uint32_t bar)
@@ -193,6 +201,46 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem,
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
                      d_tmem),
                  "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+// 1 in the one lane elect.sync picks in a converged warp, else 0
+__device__ __forceinline__ uint32_t elect_one()
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "selp.u32 %0, 1, 0, e;\n\t}"
+                 : "=r"(r));
+    return r;
+}
+// tc_mma_ss / tc_mma_ts / tc_commit issued only where `leader` is nonzero,
+// as a predicated instruction, so that a whole warp runs the issue loop
+__device__ __forceinline__ void tc_mma_ss_p(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate, uint32_t leader)
+{
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "setp.ne.b32 q, %5, 0;\n\t"
+                 "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_p(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate, uint32_t leader)
+{
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "setp.ne.b32 q, %5, 0;\n\t"
+                 "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(leader)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_commit_p(uint32_t bar, uint32_t leader)
+{
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+                 "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::"
+                 "cluster.b64 [%0];\n\t}"
+                 ::"r"(bar), "r"(leader)
                  : "memory");
 }
 

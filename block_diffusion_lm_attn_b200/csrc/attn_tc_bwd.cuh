@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto t_dp = [&](int x) { return tmem + 320 + 128 * (uint32_t)x; };
 
     KvItem it;
-    auto next_item = [&](int si, bool producer, bool &ok) -> bool {
+    auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
                 return false;
             w = item_ring[slot];
-            mbar_arrive(bar_iempty0 + 8 * slot);
+            if (arrive)
+                mbar_arrive(bar_iempty0 + 8 * slot);
         }
         if (w < 0)
             return false;
@@ -351,7 +352,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp == kBwdMmaWarp) {
         // ---------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        {
+            const uint32_t ld = elect_one();
             constexpr uint32_t idesc_s = idesc_bf16(kTcM, kBwdSub, 0);  // S^T, dP^T
             constexpr uint32_t idesc_g = idesc_bf16(kTcM, kTcD, 1);     // dV, dK
             bool ok = true;
@@ -364,18 +366,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                     const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
-                    tc_mma_ss(t_st(x), smem_desc_sw128(base + kKvSmemK + ao, 16, 1024),
-                              smem_desc_sw128(sb + bo, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    tc_mma_ss_p(t_st(x), smem_desc_sw128(base + kKvSmemK + ao, 16, 1024),
+                                smem_desc_sw128(sb + bo, 16, 1024), idesc_s, kk > 0 ? 1u : 0u,
+                                ld);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                     const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
-                    tc_mma_ss(t_dp(x), smem_desc_sw128(base + kKvSmemV + ao, 16, 1024),
-                              smem_desc_sw128(sb + kSubBytes + bo, 16, 1024), idesc_s,
-                              kk > 0 ? 1u : 0u);
+                    tc_mma_ss_p(t_dp(x), smem_desc_sw128(base + kKvSmemV + ao, 16, 1024),
+                                smem_desc_sw128(sb + kSubBytes + bo, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u, ld);
                 }
-                tc_commit(bar_sfull(x));
+                tc_commit_p(bar_sfull(x), ld);
             };
             auto issue_grad = [&](long long gg, bool first) {
                 const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
@@ -386,25 +389,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int kk = 0; kk < kBwdSub / 16; ++kk) {
                     const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bdo = smem_desc_sw128(sb + kSubBytes + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts(t_dv, t_st(x) + acol, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts_p(t_dv, t_st(x) + acol, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u,
+                                ld);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kBwdSub / 16; ++kk) {
                     const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
                     const uint64_t bq = smem_desc_sw128(sb + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts(t_dk, t_dp(x) + acol, bq, idesc_g, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts_p(t_dk, t_dp(x) + acol, bq, idesc_g, (!first || kk > 0) ? 1u : 0u,
+                                ld);
                 }
-                tc_commit(bar_empty(st));
+                tc_commit_p(bar_empty(st), ld);
             };
-            while (ok && next_item(si, false, ok)) {
-                if (!(ok = mbar_wait(bar_kvfull, (uint32_t)(si & 1), abort_flag)))
+            for (;;) {
+                const bool got = next_item(si, false, ok, lane == 0);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!got || !ok)
+                    break;
+                if (!(ok = mbar_wait_warp(bar_kvfull, (uint32_t)(si & 1), abort_flag)))
                     break;
                 tc_fence_after();
                 for (int s = 0; s <= it.nt && ok; ++s) {
                     if (s < it.nt) {
                         const long long gg = g + s;
-                        if (!(ok = mbar_wait(bar_full((int)(gg % kKvStages)),
-                                             (uint32_t)((gg / kKvStages) & 1), abort_flag)))
+                        if (!(ok = mbar_wait_warp(bar_full((int)(gg % kKvStages)),
+                                                  (uint32_t)((gg / kKvStages) & 1), abort_flag)))
                             break;
                         tc_fence_after();
                         issue_sdp(gg);
@@ -412,10 +421,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     if (s >= 1) {
                         const long long gp = g + s - 1;
                         if (s == 1 && si >= 1 &&
-                            !(ok = mbar_wait(bar_ofree, (uint32_t)((si - 1) & 1), abort_flag)))
+                            !(ok = mbar_wait_warp(bar_ofree, (uint32_t)((si - 1) & 1),
+                                                  abort_flag)))
                             break;
-                        if (!(ok = mbar_wait(bar_pfull((int)(gp & 1)), (uint32_t)((gp >> 1) & 1),
-                                             abort_flag)))
+                        if (!(ok = mbar_wait_warp(bar_pfull((int)(gp & 1)),
+                                                  (uint32_t)((gp >> 1) & 1), abort_flag)))
                             break;
                         tc_fence_after();
                         issue_grad(gp, s == 1);
@@ -423,12 +433,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(bar_kvfree);
-                tc_commit(bar_odone);
+                tc_commit_p(bar_kvfree, ld);
+                tc_commit_p(bar_odone, ld);
                 g += it.nt;
                 ++si;
             }
-            tc_commit(bar_final);
+            tc_commit_p(bar_final, ld);
             const long long c0 = clock64();
             while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
         }
@@ -653,7 +663,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fp.B = p.B; fp.Hq = p.Hq; fp.Hkv = p.Hkv; fp.L = p.L; fp.b = p.b;
     fp.qtiles = p.qtiles;
     Seg sg;
-    auto next_item = [&](int si, bool producer, bool &ok) -> bool {
+    auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -668,7 +678,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
                 return false;
             w = item_ring[slot];
-            mbar_arrive(bar_iempty0 + 8 * slot);
+            if (arrive)
+                mbar_arrive(bar_iempty0 + 8 * slot);
         }
         if (w < 0)
             return false;
@@ -728,7 +739,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else if (warp == kBwdMmaWarp) {
         // ---------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        {
+            const uint32_t ld = elect_one();
             constexpr uint32_t idesc_s = idesc_bf16(kTcM, kTcN, 0);
             constexpr uint32_t idesc_q = idesc_bf16(kTcM, kTcD, 1);
             bool ok = true;
@@ -739,17 +751,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-                    tc_mma_ss(t_s, smem_desc_sw128(base + kDqSmemQ + off, 16, 1024),
-                              smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+                    tc_mma_ss_p(t_s, smem_desc_sw128(base + kDqSmemQ + off, 16, 1024),
+                                smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u,
+                                ld);
                 }
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-                    tc_mma_ss(t_dp, smem_desc_sw128(base + kDqSmemDO + off, 16, 1024),
-                              smem_desc_sw128(kb + kTileBytes + off, 16, 1024), idesc_s,
-                              kk > 0 ? 1u : 0u);
+                    tc_mma_ss_p(t_dp, smem_desc_sw128(base + kDqSmemDO + off, 16, 1024),
+                                smem_desc_sw128(kb + kTileBytes + off, 16, 1024), idesc_s,
+                                kk > 0 ? 1u : 0u, ld);
                 }
-                tc_commit(bar_sfull);
+                tc_commit_p(bar_sfull, ld);
             };
             auto issue_dq = [&](long long jg, bool first) {
                 const uint32_t kb = base + kDqSmemRing + (uint32_t)(jg & 1) * 2 * kTileBytes;
@@ -757,36 +770,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kTcN / 16; ++kk) {
                     const uint64_t bk = smem_desc_sw128(kb + kk * 2048, kHalfTileBytes, 1024);
-                    tc_mma_ts(t_dq, t_ds(x) + kk * 8, bk, idesc_q, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts_p(t_dq, t_ds(x) + kk * 8, bk, idesc_q, (!first || kk > 0) ? 1u : 0u,
+                                ld);
                 }
-                tc_commit(bar_dsfree(x));
-                tc_commit(bar_kvempty(x));
+                tc_commit_p(bar_dsfree(x), ld);
+                tc_commit_p(bar_kvempty(x), ld);
             };
-            while (ok && next_item(si, false, ok)) {
-                if (!(ok = mbar_wait(bar_qfull, (uint32_t)(si & 1), abort_flag)))
+            for (;;) {
+                const bool got = next_item(si, false, ok, lane == 0);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!got || !ok)
+                    break;
+                if (!(ok = mbar_wait_warp(bar_qfull, (uint32_t)(si & 1), abort_flag)))
                     break;
                 for (int t = 0; t <= sg.nt && ok; ++t) {
                     const long long jg = j + t;
                     if (t < sg.nt) {
-                        if (!(ok = mbar_wait(bar_kvfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
-                                             abort_flag)))
+                        if (!(ok = mbar_wait_warp(bar_kvfull((int)(jg & 1)),
+                                                  (uint32_t)((jg >> 1) & 1), abort_flag)))
                             break;
                         // S, dP of the previous tile are in registers
-                        if (jg >= 1 && !(ok = mbar_wait(bar_sfree, (uint32_t)((jg - 1) & 1),
-                                                        abort_flag)))
+                        if (jg >= 1 && !(ok = mbar_wait_warp(bar_sfree, (uint32_t)((jg - 1) & 1),
+                                                             abort_flag)))
                             break;
                         tc_fence_after();
                         issue_sdp(jg);
                         if (t == sg.nt - 1)
-                            tc_commit(bar_qfree);
+                            tc_commit_p(bar_qfree, ld);
                     }
                     if (t >= 1) {
                         const long long jp = jg - 1;
                         if (t == 1 && si >= 1 &&
-                            !(ok = mbar_wait(bar_dqfree, (uint32_t)((si - 1) & 1), abort_flag)))
+                            !(ok = mbar_wait_warp(bar_dqfree, (uint32_t)((si - 1) & 1),
+                                                  abort_flag)))
                             break;
-                        if (!(ok = mbar_wait(bar_dsfull((int)(jp & 1)), (uint32_t)((jp >> 1) & 1),
-                                             abort_flag)))
+                        if (!(ok = mbar_wait_warp(bar_dsfull((int)(jp & 1)),
+                                                  (uint32_t)((jp >> 1) & 1), abort_flag)))
                             break;
                         tc_fence_after();
                         issue_dq(jp, t == 1);
@@ -794,11 +813,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(bar_qdone);
+                tc_commit_p(bar_qdone, ld);
                 j += sg.nt;
                 ++si;
             }
-            tc_commit(bar_final);
+            tc_commit_p(bar_final, ld);
             const long long c0 = clock64();
             while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
         }

@@ -12,7 +12,12 @@
 // Roles: warps 0-3 softmax and epilogue of tile A (thread t = row t = TMEM
 // lane t), warps 4-7 the same for tile B, warp 8 TMA producer of Q and K
 // (and the work-item fetch), warp 9 MMA issuer, warp 10 TMA producer of V,
-// warp 11 idle.  setmaxnreg moves registers from warpgroup 2 to the two
+// warp 11 idle.  All 32 lanes of warp 9 run the issue loop and its barrier
+// waits; one elected lane issues each tcgen05.mma and tcgen05.commit as a
+// predicated instruction.  (An issue loop run by one lane inside a divergent
+// branch measured about 50 cycles per MMA and per commit on the issuing side,
+// against about 19 and 3 this way, and the tensor pipe idled between
+// groups.)  setmaxnreg moves registers from warpgroup 2 to the two
 // softmax warpgroups.
 //
 // TMEM: S_A columns [0, 128), S_B [128, 256), O_A [256, 384), O_B [384, 512);
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     // Next item of this CTA, identical for every role: the Q/K producer
     // takes it from the launch's global counter and publishes it in
     // item_ring[si % 4]; the other roles read it there.
-    auto next_seg = [&](int si, bool producer, bool &ok) -> bool {
+    auto next_seg = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -170,7 +175,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
                 return false;
             w = item_ring[slot];
-            mbar_arrive(bar_iempty0 + 8 * slot);
+            if (arrive)
+                mbar_arrive(bar_iempty0 + 8 * slot);
         }
         if (w < 0)
             return false;
@@ -267,7 +273,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
     } else if (warp == 9) {
         // ---------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the loop (waits, bookkeeping); the MMAs and
+        // commits are issued by the elected lane as predicated instructions.
+        {
+            const uint32_t ld = elect_one();
             constexpr uint32_t idesc_qk = idesc_bf16(kTcM, kTcN, 0);
             constexpr uint32_t idesc_pv = idesc_bf16(kTcM, kTcD, 1);
             bool ok = true;
@@ -280,10 +289,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-                    tc_mma_ss(ts, smem_desc_sw128(qb + off, 16, 1024),
-                              smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+                    tc_mma_ss_p(ts, smem_desc_sw128(qb + off, 16, 1024),
+                                smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u,
+                                ld);
                 }
-                tc_commit(bar_sfull(x));
+                tc_commit_p(bar_sfull(x), ld);
             };
             auto issue_pv = [&](int x, long long jg, bool first) {
                 const uint32_t vb = base + kPairSmemV + (uint32_t)(jg & 1) * kTileBytes;
@@ -292,35 +302,40 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < kTcN / 16; ++kk) {
                     uint64_t bdesc = smem_desc_sw128(vb + kk * 2048, kHalfTileBytes, 1024);
-                    tc_mma_ts(to, tp + kk * 8, bdesc, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+                    tc_mma_ts_p(to, tp + kk * 8, bdesc, idesc_pv, (!first || kk > 0) ? 1u : 0u, ld);
                 }
-                tc_commit(bar_odone(x, (int)(jg & 1)));
+                tc_commit_p(bar_odone(x, (int)(jg & 1)), ld);
             };
             auto wait_k = [&](long long jg) {
-                return mbar_wait(bar_kfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1), abort_flag);
+                return mbar_wait_warp(bar_kfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
+                                      abort_flag);
             };
-            while (ok && next_seg(si, false, ok)) {
-                if (!(ok = mbar_wait(bar_qfull, (uint32_t)(si & 1), abort_flag)))
+            for (;;) {
+                const bool got = next_seg(si, false, ok, lane == 0);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!got || !ok)
+                    break;
+                if (!(ok = mbar_wait_warp(bar_qfull, (uint32_t)(si & 1), abort_flag)))
                     break;
                 if (!(ok = wait_k(j)))
                     break;
                 tc_fence_after();
                 issue_qk(0, j);
                 issue_qk(1, j);
-                tc_commit(bar_kempty((int)(j & 1)));
+                tc_commit_p(bar_kempty((int)(j & 1)), ld);
                 if (sg.nt == 1)
-                    tc_commit(bar_qfree);
+                    tc_commit_p(bar_qfree, ld);
                 for (int jj = 0; jj < sg.nt && ok; ++jj) {
                     const long long jg = j + jj;
                     const bool more = jj + 1 < sg.nt;
                     // PV_A(jg), then QK_A(jg + 1) into S_A
                     if (jj == 0 && si >= 1 &&
-                        !(ok = mbar_wait(bar_ofree(0), (uint32_t)((si - 1) & 1), abort_flag)))
+                        !(ok = mbar_wait_warp(bar_ofree(0), (uint32_t)((si - 1) & 1), abort_flag)))
                         break;
-                    if (!(ok = mbar_wait(bar_pfull(0), (uint32_t)(jg & 1), abort_flag)))
+                    if (!(ok = mbar_wait_warp(bar_pfull(0), (uint32_t)(jg & 1), abort_flag)))
                         break;
-                    if (!(ok = mbar_wait(bar_vfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
-                                         abort_flag)))
+                    if (!(ok = mbar_wait_warp(bar_vfull((int)(jg & 1)), (uint32_t)((jg >> 1) & 1),
+                                              abort_flag)))
                         break;
                     tc_fence_after();
                     issue_pv(0, jg, jj == 0);
@@ -332,24 +347,26 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     }
                     // PV_B(jg), then QK_B(jg + 1) into S_B
                     if (jj == 0 && si >= 1 &&
-                        !(ok = mbar_wait(bar_ofree(1), (uint32_t)((si - 1) & 1), abort_flag)))
+                        !(ok = mbar_wait_warp(bar_ofree(1), (uint32_t)((si - 1) & 1), abort_flag)))
                         break;
-                    if (!(ok = mbar_wait(bar_pfull(1), (uint32_t)(jg & 1), abort_flag)))
+                    if (!(ok = mbar_wait_warp(bar_pfull(1), (uint32_t)(jg & 1), abort_flag)))
                         break;
                     tc_fence_after();
                     issue_pv(1, jg, jj == 0);
-                    tc_commit(bar_vempty((int)(jg & 1)));
+                    tc_commit_p(bar_vempty((int)(jg & 1)), ld);
                     if (more) {
                         issue_qk(1, jg + 1);
-                        tc_commit(bar_kempty((int)((jg + 1) & 1)));
+                        tc_commit_p(bar_kempty((int)((jg + 1) & 1)), ld);
                         if (jj + 2 == sg.nt)
-                            tc_commit(bar_qfree);
+                            tc_commit_p(bar_qfree, ld);
                     }
                 }
+                if (!ok)
+                    break;
                 j += sg.nt;
                 ++si;
             }
-            tc_commit(bar_final);
+            tc_commit_p(bar_final, ld);
             const long long c0 = clock64();
             while (!mbar_try_wait(bar_final, 0) && clock64() - c0 < kWaitCycles) {}
         }
