@@ -118,6 +118,32 @@ def decode_inputs_for(s: DecodeShape):
                          len_range=(s.len_lo, s.len_hi), seed=s.seed)
 
 
+def fwd_sample_rows(B: int, H: int, L: int, b: int, n: int, heads: int = 8,
+                    per_block: int = 16, seed: int = 1):
+    """Flat row ids of a [B, H, 2L] forward output for a sampled parity check
+    (sorted, unique): in ``heads`` seeded (batch, head) pairs -- the first and
+    the last always among them -- rows of the first and the last block of
+    each half (the whole block when b <= per_block, else ``per_block`` rows
+    spread over it, its first and last row included), plus ``n`` uniform
+    picks over the whole tensor."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    nh = B * H
+    if nh <= heads:
+        hsel = torch.arange(nh)
+    else:
+        mid = torch.randperm(nh - 2, generator=g)[:heads - 2] + 1
+        hsel = torch.cat([torch.tensor([0, nh - 1]), mid])
+    if b <= per_block:
+        inblk = torch.arange(b)
+    else:
+        inblk = torch.linspace(0, b - 1, per_block).round().long().unique()
+    starts = torch.tensor([0, L - b, L, 2 * L - b])
+    local = (starts[:, None] + inblk[None, :]).reshape(-1)
+    forced = (hsel[:, None] * (2 * L) + local[None, :]).reshape(-1)
+    pick = torch.randint(0, nh * 2 * L, (n,), generator=g)
+    return torch.unique(torch.cat([pick, forced])).tolist()
+
+
 def sample_rows(total_rows: int, block: int, n: int, seed: int = 1):
     """A seeded sample of flat row ids that always includes the first and
     last ``block`` rows plus ``n`` uniform picks (sorted, unique)."""

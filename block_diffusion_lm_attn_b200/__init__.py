@@ -173,6 +173,15 @@ def bd_attn_debug_fwd_kernel(Hq, Hkv, d):
     return fn(Hq, Hkv, d)
 
 
+def bd_attn_debug_reset_sched():
+    """Test hook (include/bd_attn_debug.h): synchronise the device and zero
+    every work-counter pair of the persistent kernels."""
+    fn = load().bd_attn_debug_reset_sched
+    fn.restype = ctypes.c_int
+    fn.argtypes = []
+    return fn()
+
+
 def bd_attn_debug_set_grid(ctas):
     """Test hook (include/bd_attn_debug.h): cap the grid of the persistent
     head-dim-128 kernels at `ctas` CTAs (0 restores one CTA per SM)."""

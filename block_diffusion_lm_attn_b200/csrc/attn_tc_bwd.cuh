@@ -246,6 +246,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
                                              (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
                 return false;
+            if (si == 0)
+                sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < kv_items(p) ? (int)t : -1;
             item_ring[slot] = w;
@@ -335,12 +337,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
         if (lane == 0) {
-            __threadfence();
-            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
-                g_sched_next[p.sched_slot] = 0;
-                g_sched_done[p.sched_slot] = 0;
-                __threadfence();
-            }
+            sched_finish(p.sched_slot);
             const long long c0 = clock64();
             auto drain = [&](uint32_t bar, uint32_t par) {
                 while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}
@@ -670,6 +667,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
                                              (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
                 return false;
+            if (si == 0)
+                sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < FwdSource::items(fp) ? (int)t : -1;
             item_ring[slot] = w;
@@ -722,12 +721,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     iss = g + 1;
                 }
             }
-            __threadfence();
-            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
-                g_sched_next[p.sched_slot] = 0;
-                g_sched_done[p.sched_slot] = 0;
-                __threadfence();
-            }
+            sched_finish(p.sched_slot);
             const long long c0 = clock64();
             auto drain = [&](uint32_t bar, uint32_t par) {
                 while (!mbar_try_wait(bar, par) && clock64() - c0 < kWaitCycles) {}

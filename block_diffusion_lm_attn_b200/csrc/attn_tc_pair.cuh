@@ -167,6 +167,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
                                              (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
                 return false;
+            if (si == 0)
+                sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < pair_items(p) ? (int)t : -1;
             item_ring[slot] = w;
@@ -227,12 +229,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
             }
             // this CTA takes no more items; the last CTA resets the pair
-            __threadfence();
-            if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
-                g_sched_next[p.sched_slot] = 0;
-                g_sched_done[p.sched_slot] = 0;
-                __threadfence();
-            }
+            sched_finish(p.sched_slot);
             // wait (bounded) for every copy this role issued
             const long long c0 = clock64();
             auto drain = [&](uint32_t bar, uint32_t par) {

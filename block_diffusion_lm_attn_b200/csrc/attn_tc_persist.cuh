@@ -95,6 +95,30 @@ constexpr int kSchedSlots = 64;
 __device__ int g_fault_skip_k;
 __device__ unsigned int g_sched_next[kSchedSlots];
 __device__ unsigned int g_sched_done[kSchedSlots];
+__device__ unsigned int g_sched_claim[kSchedSlots];
+
+// Called once per CTA before its first fetch from counter pair `slot`.
+// More claims than the launch has CTAs means that another launch uses the
+// pair at the same time (the two then share the item counter and compute
+// wrong results): that is recorded in the device status word.
+__device__ __forceinline__ void sched_claim(int slot)
+{
+    if (atomicAdd(&g_sched_claim[slot], 1u) >= gridDim.x)
+        raise_device_code(DEV_SCHED_OVERLAP);
+}
+
+// Called once per CTA after its last fetch: the launch's last CTA resets the
+// pair for the next launch that draws it.
+__device__ __forceinline__ void sched_finish(int slot)
+{
+    __threadfence();
+    if (atomicAdd(&g_sched_done[slot], 1u) == gridDim.x - 1) {
+        g_sched_next[slot] = 0;
+        g_sched_done[slot] = 0;
+        g_sched_claim[slot] = 0;
+        __threadfence();
+    }
+}
 
 struct FwdSource {
     __device__ void init(const PParams &) {}
@@ -338,6 +362,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (si >= 4 && !(ok = mbar_wait(bar_iempty0 + 8 * slot,
                                              (uint32_t)(((si - 4) >> 2) & 1), abort_flag)))
                 return false;
+            if (si == 0)
+                sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < FwdSource::items(p) ? (int)t : -1;
             item_ring[slot] = w;
@@ -397,12 +423,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             if (KIND == 0) {
                 // this CTA takes no more items; the last CTA resets the pair
-                __threadfence();
-                if (atomicAdd(&g_sched_done[p.sched_slot], 1u) == gridDim.x - 1) {
-                    g_sched_next[p.sched_slot] = 0;
-                    g_sched_done[p.sched_slot] = 0;
-                    __threadfence();
-                }
+                sched_finish(p.sched_slot);
             }
             // wait (bounded) for every copy this role issued
             const long long c0 = clock64();

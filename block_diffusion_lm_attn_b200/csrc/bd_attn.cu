@@ -711,6 +711,18 @@ bd_status bd_attn_debug_set_grid(int ctas)
     return BD_OK;
 }
 
+bd_status bd_attn_debug_reset_sched(void)
+{
+    unsigned int zero[bd::kSchedSlots] = {};
+    if (cudaDeviceSynchronize() != cudaSuccess)
+        return BD_ERR_CUDA;
+    return (cudaMemcpyToSymbol(bd::g_sched_next, zero, sizeof zero) == cudaSuccess &&
+            cudaMemcpyToSymbol(bd::g_sched_done, zero, sizeof zero) == cudaSuccess &&
+            cudaMemcpyToSymbol(bd::g_sched_claim, zero, sizeof zero) == cudaSuccess)
+               ? BD_OK
+               : BD_ERR_CUDA;
+}
+
 bd_status bd_attn_get_device_status(cudaStream_t stream)
 {
     if (cudaStreamSynchronize(stream) != cudaSuccess)

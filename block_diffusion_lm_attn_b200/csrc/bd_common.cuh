@@ -15,6 +15,7 @@ __device__ unsigned int g_status_word;
 enum DeviceCode : unsigned int {
     DEV_BAD_CACHE_LEN = 1u,
     DEV_WAIT_TIMEOUT = 2u,
+    DEV_SCHED_OVERLAP = 4u, // two launches shared a work counter pair
 };
 
 __device__ __forceinline__ void raise_device_code(unsigned int code)

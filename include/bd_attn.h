@@ -45,8 +45,9 @@ typedef enum {
     BD_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size or mode */
     BD_ERR_UNSUPPORTED = 2,     /* valid request this build does not handle */
     BD_ERR_CUDA = 3,            /* a CUDA runtime/driver call failed */
-    BD_ERR_DEVICE_TIMEOUT = 4   /* a bounded device wait ran out, or a
-                                   device-side range check failed */
+    BD_ERR_DEVICE_TIMEOUT = 4   /* a bounded device wait ran out, a
+                                   device-side range check failed, or two
+                                   launches shared a work counter pair */
 } bd_status;
 
 /*
@@ -83,7 +84,11 @@ typedef enum {
  * round-robin when the call is made (and so fixed inside a captured CUDA
  * graph) and reset by the launch's last CTA.  Launches sharing a pair must
  * not overlap in time: keep fewer than 64 calls in flight per device, and do
- * not run two replays of one captured graph at the same time.
+ * not run two replays of one captured graph at the same time.  Each CTA
+ * counts itself into the pair before its first fetch; a count beyond the
+ * launch's own CTAs means such an overlap, and the device status word then
+ * records BD_ERR_DEVICE_TIMEOUT (the outputs of the overlapping launches are
+ * unreliable).
  */
 BD_API bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
                       float *lse, int B, int Hq, int Hkv, int L, int b, int d,
@@ -356,7 +361,8 @@ BD_API size_t bd_attn_decode_workspace_bytes(int B, int Hq, int Hkv, int b, int 
 
 /* Synchronises `stream`, then returns and clears the device status word of
  * the current device: BD_OK, or BD_ERR_DEVICE_TIMEOUT if a kernel gave up a
- * bounded wait or rejected a device-resident size since the last call;
+ * bounded wait, rejected a device-resident size, or found its work counter
+ * pair in use by another launch since the last call;
  * BD_ERR_CUDA if the synchronisation itself failed. */
 BD_API bd_status bd_attn_get_device_status(struct CUstream_st *stream);
 

@@ -1,7 +1,7 @@
 /*
  * bd_attn_debug.h -- test hooks of libbdattn.so (no counterpart on the
- * source pages): the failure-detection path, and the grid size of the
- * persistent kernels.
+ * source pages): the failure-detection path, the grid size of the
+ * persistent kernels, the forward kernel selected, and the work counters.
  *
  * Every wait inside the tensor-core kernels is bounded: when one runs out,
  * the kernel records BD_ERR_DEVICE_TIMEOUT in the device status word (read
@@ -50,6 +50,15 @@ BD_API bd_status bd_attn_debug_set_grid(int ctas);
  * Needs the CUDA runtime (it reads the compiled kernel's attributes).
  */
 BD_API int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d);
+
+/*
+ * Synchronises the current device, then zeroes every work-counter pair of
+ * the persistent kernels (item counter, finished-CTA counter, claim
+ * counter).  For tests that run overlapping launches on one pair on
+ * purpose: the pair's counts are then mixed, and its next user would take
+ * wrong items.  Returns BD_OK or BD_ERR_CUDA.
+ */
+BD_API bd_status bd_attn_debug_reset_sched(void);
 
 #ifdef __cplusplus
 }

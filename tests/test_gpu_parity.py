@@ -120,8 +120,8 @@ def test_fwd_other_scale_and_value_ranges():
 def _fwd_sampled(s, nsample):
     q, k, v = bd_inputs.fwd_inputs_for(s)
     out, lse = run_fwd(q, k, v, s.L, s.b, s.scale)
-    total = s.B * s.Hq * 2 * s.L
-    rows = bd_inputs.sample_rows(total, 2 * s.b + 1, nsample)
+    # every sampled head contributes the first and last block of each half
+    rows = bd_inputs.fwd_sample_rows(s.B, s.Hq, s.L, s.b, nsample)
     ro, rl = oracle.fwd(q, k, v, s.L, s.b, s.scale, rows=rows)
     d = s.d
     o = out.reshape(-1, d)[torch.tensor(rows, device=out.device)]
