@@ -62,8 +62,12 @@ KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
                   "attn_mma.cuh", "bd_common.cuh")
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
-    "bd_tc_pair_kernel": (None, None, None),
-    "bd_tc_persist_kernel<1>": (None, None, None),
+    "bd_tc_pair_kernel": (
+        301549824, "9edd8f12e5931c23",
+        "ncu, training-shape forward, 4th launch of `bench.py --only fwd`"),
+    "bd_tc_persist_kernel<1>": (
+        543778776, "9edd8f12e5931c23",
+        "ncu, denoise decode, median of 5 launches of `bench.py --only decode`"),
 }
 
 
