@@ -90,6 +90,9 @@ __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
     sg.nt = sg.n0 + n1;
 }
 
+// DH: head dim of the tensors, 128, or 64 read zero-extended to 128 columns
+// (the QKs skip the zero half; the upper 64 columns of O are never written).
+template <int DH>
 __global__ void __launch_bounds__(kPairThreads, 1)
     bd_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -285,6 +288,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 const uint32_t ts = tmem + (uint32_t)x * 128;
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    if (kk * 16 >= DH) // zero columns of a head dim of 64
+                        break;
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                     tc_mma_ss_p(ts, smem_desc_sw128(qb + off, 16, 1024),
                                 smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u,
@@ -436,6 +441,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const uint32_t epi = base + kPairSmemEpi + (uint32_t)warp * (32 * 128);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                if (h * 64 >= DH) // O columns past the head dim are not output
+                    break;
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int q4 = 2 * h + q;
@@ -467,7 +474,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                  : "memory");
                     const int trow = wq * 32 + r;
                     if (trow < sg.nrows)
-                        reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * kTcD)[h * 8 + cc] =
+                        reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * DH)[h * 8 + cc] =
                             make_uint4(x0, x1, x2, x3);
                 }
                 __syncwarp();

@@ -40,6 +40,7 @@ struct PParams {
                      // {rows (0: none), CTA of its last tile, out row, 0}
     const int32_t *cache_len;
     int B, Hq, Hkv, L, b;
+    int d;         // head dim of q, k, v, out: 128, or 64 (read zero-extended to 128)
     int nkeys;     // key rows per kv-head: 2L or S_cap
     int mode;      // decode: 0 bidirectional, 1 causal
     int qtiles;    // fwd: 128-row query tiles per half
@@ -256,7 +257,10 @@ struct DecSource {
 
 // ----------------------------------------------------------------------------
 
-template <int KIND>
+// KIND 0: training/prefill form, 1: block decode.  DH: head dim of the
+// tensors, 128, or 64 read zero-extended to 128 columns (the QKs skip the zero
+// half; the upper 64 columns of O are computed but never written out).
+template <int KIND, int DH>
 __global__ void __launch_bounds__(kTcThreads, 1)
     bd_tc_persist_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -526,6 +530,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t ts = t_s0 + (uint32_t)b * 128;
 #pragma unroll
                     for (int kk = 0; kk < kTcD / 16; ++kk) {
+                        if (kk * 16 >= DH) // zero columns of a head dim of 64
+                            break;
                         const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                         tc_mma_ss(ts, smem_desc_sw128(qb + off, 16, 1024),
                                   smem_desc_sw128(kb + off, 16, 1024), idesc_qk,
@@ -632,6 +638,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t epi = base + kSmemEpi + (uint32_t)warp * (32 * 256);
 #pragma unroll
             for (int q4 = 0; q4 < kTcD / 32; ++q4) {
+                if (q4 * 32 >= DH) // O columns past the head dim are not output
+                    break;
                 uint32_t o[32];
                 tmem_ld32(t_o + lane_off + q4 * 32, o);
                 tmem_wait_ld();
@@ -648,7 +656,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                      : "memory");
                     }
                 } else if (valid && to_out) {
-                    uint4 *orow = reinterpret_cast<uint4 *>(p.out + grow * kTcD);
+                    uint4 *orow = reinterpret_cast<uint4 *>(p.out + grow * DH);
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         uint4 v4;
@@ -679,8 +687,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                  : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
                                  : "r"(epi + (uint32_t)r * 256 + ((cc ^ (uint32_t)(r & 7)) << 4))
                                  : "memory");
-                    if (warp * 32 + r < sg.nrows)
-                        reinterpret_cast<uint4 *>(p.out + (row0 + r) * kTcD)[cc] =
+                    if (warp * 32 + r < sg.nrows && (int)cc * 8 < DH)
+                        reinterpret_cast<uint4 *>(p.out + (row0 + r) * DH)[cc] =
                             make_uint4(x0, x1, x2, x3);
                 }
                 __syncwarp();
@@ -742,8 +750,8 @@ __global__ void __launch_bounds__(256)
             const float lfill = tiles < 0 ? NAN : -INFINITY;
             for (int r = threadIdx.x; r < p.Hq * p.b; r += blockDim.x) {
                 const size_t orow = (size_t)i * p.Hq * p.b + r;
-                for (int t = 0; t < kTcD; ++t)
-                    p.out[orow * kTcD + t] = __float2bfloat16_rn(fill);
+                for (int t = 0; t < p.d; ++t)
+                    p.out[orow * p.d + t] = __float2bfloat16_rn(fill);
                 p.lse[orow] = lfill;
             }
             if (threadIdx.x == 0 && tiles < 0)
@@ -797,7 +805,8 @@ __global__ void __launch_bounds__(256)
         uint2 o2;
         o2.x = pack_bf16x2(acc[k].x * inv, acc[k].y * inv);
         o2.y = pack_bf16x2(acc[k].z * inv, acc[k].w * inv);
-        reinterpret_cast<uint2 *>(p.out + orow * kTcD)[lane] = o2;
+        if (lane * 4 < p.d)
+            reinterpret_cast<uint2 *>(p.out + orow * p.d)[lane] = o2;
         if (lane == 0)
             p.lse[orow] = z[k] > 0.f ? m[k] + __logf(z[k]) : -INFINITY;
     }

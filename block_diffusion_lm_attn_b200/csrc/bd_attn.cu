@@ -48,13 +48,14 @@ inline size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 // setmaxnreg, which can only hand out what the CTA was launched with: use it
 // only if the compiled kernel's per-thread registers cover the split (a
 // warpgroup asking for more than exists would wait for ever).
+template <int DH>
 bool pair_kernel_usable()
 {
     static std::atomic<int> usable{-1};
     int u = usable.load();
     if (u < 0) {
         cudaFuncAttributes a;
-        u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel) == cudaSuccess &&
+        u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel<DH>) == cudaSuccess &&
              (long long)a.numRegs * bd::kPairThreads >=
                  2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther)
                 ? 1
@@ -62,6 +63,11 @@ bool pair_kernel_usable()
         usable.store(u);
     }
     return u == 1;
+}
+
+bool pair_kernel_usable(int d)
+{
+    return d == 64 ? pair_kernel_usable<64>() : pair_kernel_usable<128>();
 }
 
 // Grid cap set by bd_attn_debug_set_grid (0: none).
@@ -82,9 +88,10 @@ int persistent_grid()
 
 // Decode launch plan.  A pure function of the sizes, so the workspace query
 // and the launch agree without a device round trip.
-//   d = 128: stream-K over (unit, key tile) on <= kMaxGrid persistent CTAs;
-//            scratch = 2 partial (o, lse) slots of 128 rows per CTA.
-//   d < 128: split-KV with `nsplit` chunks of `chunk` keys per (sequence,
+//   d = 128 or 64: stream-K over (unit, key tile) on <= kMaxGrid persistent
+//            CTAs (d = 64 on tiles zero-extended to 128 columns); scratch =
+//            2 partial (o, lse) slots of 128 rows x 128 columns per CTA.
+//   d = 32:  split-KV with `nsplit` chunks of `chunk` keys per (sequence,
 //            kv-head, 64-row tile); scratch = nsplit partials per row.
 struct DecodePlan {
     bool tc;
@@ -100,7 +107,7 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
         return false;
     const long long rows = (long long)(Hq / Hkv) * b;
     pl.rows_all = (size_t)B * Hq * b;
-    pl.tc = (d == 128);
+    pl.tc = (d == 128 || d == 64);
     if (pl.tc) {
         pl.row_tiles = (int)cdiv(rows, bd::kTcM);
         pl.nsplit = 0;
@@ -195,13 +202,16 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 // 3-D map over a row-major bf16 tensor [n2][n1][128]: boxes of 64 columns x
 // box_rows rows x 1, 128-byte swizzle, rows beyond n1 read as zero.
 bool make_map_rows(CUtensorMap *m, const void *base, uint64_t n1, uint64_t n2,
-                   uint32_t box_rows)
+                   uint32_t box_rows, uint64_t d = 128)
 {
     auto enc = tensor_map_encoder();
     if (!enc)
         return false;
-    cuuint64_t dims[3] = {128, n1, n2};
-    cuuint64_t strides[2] = {128 * 2, 128 * 2 * n1};
+    // rows of d bf16 (d = 64 or 128) read as 64-column boxes; with d = 64 the
+    // box at column 64 lies wholly outside the tensor and reads as zeros, so
+    // the head-dim-128 kernels run unchanged on a zero-extended tile
+    cuuint64_t dims[3] = {d, n1, n2};
+    cuuint64_t strides[2] = {d * 2, d * 2 * n1};
     cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
@@ -213,9 +223,9 @@ bool make_map_rows(CUtensorMap *m, const void *base, uint64_t n1, uint64_t n2,
 }
 
 bool make_map_rows128(CUtensorMap *m, const void *base, uint64_t n1,
-                      uint64_t n2)
+                      uint64_t n2, uint64_t d = 128)
 {
-    return make_map_rows(m, base, n1, n2, 128);
+    return make_map_rows(m, base, n1, n2, 128, d);
 }
 
 // Counter pair of the next persistent launch that hands out work items
@@ -226,16 +236,35 @@ int next_sched_slot()
     return (int)(g_launches.fetch_add(1u) % bd::kSchedSlots);
 }
 
+template <int KIND, int DH>
+bd_status launch_persist_dh(const CUtensorMap &mq, const CUtensorMap &mk,
+                            const CUtensorMap &mv, const bd::PParams &p, int grid,
+                            cudaStream_t st)
+{
+    auto kern = bd::bd_tc_persist_kernel<KIND, DH>;
+    if (set_smem<bd::bd_tc_persist_kernel<KIND, DH>>(bd::kTcSmemBytes) != BD_OK)
+        return BD_ERR_CUDA;
+    kern<<<grid, bd::kTcThreads, bd::kTcSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+template <int DH>
+bd_status launch_pair(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                      const bd::PParams &p, int grid, cudaStream_t st)
+{
+    if (set_smem<bd::bd_tc_pair_kernel<DH>>(bd::kPairSmemBytes) != BD_OK)
+        return BD_ERR_CUDA;
+    bd::bd_tc_pair_kernel<DH><<<grid, bd::kPairThreads, bd::kPairSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
 template <int KIND>
 bd_status launch_persist(const CUtensorMap &mq, const CUtensorMap &mk,
                          const CUtensorMap &mv, const bd::PParams &p, int grid,
                          cudaStream_t st)
 {
-    auto kern = bd::bd_tc_persist_kernel<KIND>;
-    if (set_smem<bd::bd_tc_persist_kernel<KIND>>(bd::kTcSmemBytes) != BD_OK)
-        return BD_ERR_CUDA;
-    kern<<<grid, bd::kTcThreads, bd::kTcSmemBytes, st>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+    return p.d == 64 ? launch_persist_dh<KIND, 64>(mq, mk, mv, p, grid, st)
+                     : launch_persist_dh<KIND, 128>(mq, mk, mv, p, grid, st);
 }
 
 template <int D>
@@ -319,15 +348,16 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
                                               pl.lse_bytes);
         p.cache_len = cache_len;
         p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
+        p.d = d;
         p.nkeys = S_cap;
         p.mode = mode;
         p.row_tiles = pl.row_tiles;
         p.rows_unit = (Hq / Hkv) * b;
         p.scale_log2 = scale_log2;
         CUtensorMap mq, mk, mv;
-        if (!make_map_rows128(&mq, q_blk, (uint64_t)p.rows_unit, (uint64_t)B * Hkv) ||
-            !make_map_rows128(&mk, k_cache, (uint64_t)S_cap, (uint64_t)B * Hkv) ||
-            !make_map_rows128(&mv, v_cache, (uint64_t)S_cap, (uint64_t)B * Hkv))
+        if (!make_map_rows128(&mq, q_blk, (uint64_t)p.rows_unit, (uint64_t)B * Hkv, d) ||
+            !make_map_rows128(&mk, k_cache, (uint64_t)S_cap, (uint64_t)B * Hkv, d) ||
+            !make_map_rows128(&mv, v_cache, (uint64_t)S_cap, (uint64_t)B * Hkv, d))
             return BD_ERR_CUDA;
         const int G = persistent_grid();
         bd_status st = launch_persist<1>(mq, mk, mv, p, G, stream);
@@ -407,34 +437,32 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
     if ((long long)B * Hq > 65535LL || 2LL * L * (long long)B * Hq * d > (1LL << 40))
         return BD_ERR_UNSUPPORTED;
 
-    if (d == 128) {
+    if (d == 128 || d == 64) {
+        // tcgen05 kernels; d = 64 runs on tiles zero-extended to 128 columns
         bd::PParams p = {};
         p.out = static_cast<bf16 *>(out);
         p.lse = lse;
         p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
+        p.d = d;
         p.nkeys = 2 * L;
         p.qtiles = (int)cdiv(L, bd::kTcM);
         p.scale_log2 = scale * bd::kLog2e;
         CUtensorMap mq, mk, mv;
         const uint64_t N = 2ull * L;
-        if (!make_map_rows128(&mq, q, N, (uint64_t)B * Hq) ||
-            !make_map_rows128(&mk, k, N, (uint64_t)B * Hkv) ||
-            !make_map_rows128(&mv, v, N, (uint64_t)B * Hkv))
+        if (!make_map_rows128(&mq, q, N, (uint64_t)B * Hq, d) ||
+            !make_map_rows128(&mk, k, N, (uint64_t)B * Hkv, d) ||
+            !make_map_rows128(&mv, v, N, (uint64_t)B * Hkv, d))
             return BD_ERR_CUDA;
         p.sched_slot = next_sched_slot();
         // two query heads of one GQA group per CTA when the group size is even
-        const bool pair = (Hq / Hkv) % 2 == 0 && pair_kernel_usable();
+        const bool pair = (Hq / Hkv) % 2 == 0 && pair_kernel_usable(d);
         const long long items = (long long)B * (pair ? Hq / 2 : Hq) * 2 * p.qtiles;
         int G = persistent_grid();
         if (items < G)
             G = (int)items;
-        if (pair) {
-            if (set_smem<bd::bd_tc_pair_kernel>(bd::kPairSmemBytes) != BD_OK)
-                return BD_ERR_CUDA;
-            bd::bd_tc_pair_kernel<<<G, bd::kPairThreads, bd::kPairSmemBytes, stream>>>(mq, mk,
-                                                                                     mv, p);
-            return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
-        }
+        if (pair)
+            return d == 64 ? launch_pair<64>(mq, mk, mv, p, G, stream)
+                           : launch_pair<128>(mq, mk, mv, p, G, stream);
         return launch_persist<0>(mq, mk, mv, p, G, stream);
     }
 
@@ -698,9 +726,9 @@ int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d)
 {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !supported_d(d))
         return -1;
-    if (d != 128)
+    if (d == 32)
         return 0;
-    return ((Hq / Hkv) % 2 == 0 && pair_kernel_usable()) ? 2 : 1;
+    return ((Hq / Hkv) % 2 == 0 && pair_kernel_usable(d)) ? 2 : 1;
 }
 
 bd_status bd_attn_debug_set_grid(int ctas)

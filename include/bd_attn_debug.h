@@ -21,7 +21,7 @@ extern "C" {
 
 /*
  * Arms a one-shot fault on the current device: in the next launch of the
- * head-dim-128 kernel (bd_attn_fwd or bd_attn_decode with d = 128), CTA 0
+ * tcgen05 kernel (bd_attn_fwd or bd_attn_decode with d = 128 or 64), CTA 0
  * skips the copy of its first K tile, so the wait for that tile runs out
  * after about two seconds and the launch reports BD_ERR_DEVICE_TIMEOUT.
  * The outputs of that launch are undefined; later launches are unaffected.
@@ -31,8 +31,8 @@ extern "C" {
 BD_API bd_status bd_attn_debug_inject_fault(int kind);
 
 /*
- * Caps the grid of the persistent head-dim-128 kernels (bd_attn_fwd and
- * bd_attn_decode with d = 128) at `ctas` CTAs for every later launch from
+ * Caps the grid of the persistent tcgen05 kernels (bd_attn_fwd and
+ * bd_attn_decode with d = 128 or 64) at `ctas` CTAs for every later launch from
  * any thread, so tests can run the forward's dynamic hand-out and the
  * decode's stream-K split and combine at grid sizes other than one CTA per
  * SM.  ctas = 0 restores the default (one CTA per SM, at most 148).
@@ -43,10 +43,10 @@ BD_API bd_status bd_attn_debug_set_grid(int ctas);
 
 /*
  * Which kernel bd_attn_fwd runs for these sizes on the current device:
- * 2 = tcgen05 kernel with two query heads of a GQA group per CTA (d = 128,
- * even group size), 1 = tcgen05 kernel with one query tile per CTA (d = 128,
- * odd group size, or the paired kernel's register split unavailable),
- * 0 = mma.sync kernel (d = 32, 64), -1 = sizes bd_attn_fwd rejects.
+ * 2 = tcgen05 kernel with two query heads of a GQA group per CTA (d = 128
+ * or 64, even group size), 1 = tcgen05 kernel with one query tile per CTA
+ * (d = 128 or 64, odd group size, or the paired kernel's register split
+ * unavailable), 0 = mma.sync kernel (d = 32), -1 = sizes bd_attn_fwd rejects.
  * Needs the CUDA runtime (it reads the compiled kernel's attributes).
  */
 BD_API int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d);

@@ -84,18 +84,22 @@ FWD_GRID = [
     (1, 1, 1, 64, 8, 128),      # fewer work items than SMs
     (3, 2, 2, 136, 17, 128),    # ragged query tiles in both halves
     (1, 4, 1, 512, 512, 128),   # one block per half (b = L)
+    (1, 4, 2, 200, 8, 64),      # head dim 64 on the paired kernel, ragged tails
+    (2, 3, 3, 136, 17, 64),     # head dim 64 on the one-tile kernel
 ]
 
 
 def test_fwd_kernel_selection():
-    """Even GQA groups of head dim 128 run the paired tcgen05 kernel (the
-    one the benchmark times), odd groups the one-tile tcgen05 kernel, head
-    dims 32 and 64 the mma.sync kernel; so the grid below covers each."""
+    """Even GQA groups of head dim 128 or 64 run the paired tcgen05 kernel
+    (the one the benchmark times), odd groups the one-tile tcgen05 kernel,
+    head dim 32 the mma.sync kernel; so the grid below covers each."""
     assert bd.bd_attn_debug_fwd_kernel(32, 8, 128) == 2
     assert bd.bd_attn_debug_fwd_kernel(4, 2, 128) == 2
     assert bd.bd_attn_debug_fwd_kernel(8, 8, 128) == 1
     assert bd.bd_attn_debug_fwd_kernel(3, 1, 128) == 1
-    assert bd.bd_attn_debug_fwd_kernel(2, 2, 64) == 0
+    assert bd.bd_attn_debug_fwd_kernel(4, 2, 64) == 2
+    assert bd.bd_attn_debug_fwd_kernel(2, 2, 64) == 1
+    assert bd.bd_attn_debug_fwd_kernel(2, 2, 32) == 0
     assert bd.bd_attn_debug_fwd_kernel(3, 2, 128) == -1
 
 
@@ -172,6 +176,7 @@ DEC_GRID = [
     (1, 2, 1, 200, 128, [300], 1),       # b > 128: rows with no key in a piece
     (2, 4, 4, 3, 128, [20000, 1], 0),    # one long unit cut across many CTAs
     (5, 8, 2, 7, 128, [0, 128, 129, 1023, 8000], 1),
+    (3, 8, 2, 16, 64, [2, 600, 20000], 0),       # head dim 64, one unit cut across CTAs
 ]
 
 
@@ -300,8 +305,8 @@ def test_internal_workspace_survives_growth_under_a_captured_graph():
         with torch.cuda.graph(g, stream=s):
             bd.decode(qd, kd, vd, cd, 0, out=out, lse=lse, stream=s)
     torch.cuda.synchronize()
-    # a head-dim-64 call whose split-KV scratch exceeds the current buffer
-    B2, Hq2, Hkv2, b2, d2 = 128, 32, 8, 32, 64
+    # a head-dim-32 call whose split-KV scratch exceeds the current buffer
+    B2, Hq2, Hkv2, b2, d2 = 256, 32, 8, 32, 32
     assert (bd.workspace_bytes(B2, Hq2, Hkv2, b2, d2, 64) >
             bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap))
     q2, kc2, vc2, cl2 = bd_inputs.decode_inputs(B2, Hq2, Hkv2, b2, d2, 64,

@@ -2,8 +2,9 @@
 that cannot allocate device memory at decode time (its split-KV scratch is a
 fixed array inside the library).  Two calls in a row, with different inputs,
 each compared with bd_attn_decode on the same inputs, and once directly with
-the fp64 oracle; both head-dim paths (the d = 128 stream-K layout and the
-d = 64 split-KV layout share the array); and a call inside a captured CUDA
+the fp64 oracle; both scratch layouts (the stream-K layout of the tcgen05
+kernel, d = 128 and 64, and the split-KV layout of the d = 32 kernel share
+the array); and a call inside a captured CUDA
 graph in global capture mode, where any allocation would fail the capture.
 Collected last so that a run stopping at the first failure has already run
 every other test."""
@@ -46,6 +47,7 @@ CASES = [
     (8, 32, 8, 28, 128, [513, 4000, 77, 1024, 3001, 900, 12, 2500], 1),
     (4, 8, 2, 16, 64, [300, 5, 1200, 64], 0),
     (3, 4, 4, 8, 64, [100, 0, 40], 1),
+    (3, 8, 2, 16, 32, [700, 3, 64], 0),
 ]
 
 
@@ -67,7 +69,7 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
         _compare(ref_o, ref_l, out, lse)
 
     # a size whose scratch exceeds the fixed array is refused up front
-    B, Hq, Hkv, b, d, S_cap = 256, 64, 8, 32, 64, 65536
+    B, Hq, Hkv, b, d, S_cap = 256, 64, 8, 32, 32, 65536
     assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) > SCRATCH_MAX
     A = 1 << 20
     st = bd.bd_attn_decode_noalloc(A, A, A, A, A, A, B, Hq, Hkv, b, d, 0,
