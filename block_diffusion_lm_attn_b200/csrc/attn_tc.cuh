@@ -429,37 +429,6 @@ __device__ __forceinline__ void softmax_p_tile(const float *s, float sl2,
     }
 }
 
-// As softmax_p_tile for a tile in which only the 32-column words set in
-// `live` (the same for every lane of the warp) hold a visible key for some row
-// of the warp: the other words get P = 0 without any exponential.
-__device__ __forceinline__ void softmax_p_tile_live(const float *s, float sl2,
-                                                    float nm, uint32_t ts,
-                                                    float *rsum, uint32_t live)
-{
-#pragma unroll
-    for (int c4 = 0; c4 < kTcN / 32; ++c4) {
-        uint32_t pk[16];
-        if ((live >> c4) & 1u) {
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                float x0, x1;
-                const int b0 = c4 * 32 + c;
-                ffma2(x0, x1, s[b0], s[b0 + 1], sl2, sl2, nm, nm);
-                x0 = ex2(x0);
-                x1 = ex2(x1);
-                const int a = (c >> 1) & 1;
-                fadd2(rsum[2 * a], rsum[2 * a + 1], rsum[2 * a], rsum[2 * a + 1], x0, x1);
-                pk[c / 2] = pack_bf16x2(x0, x1);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                pk[i] = 0u;
-        }
-        tmem_st16(ts + c4 * 16, pk);
-    }
-}
-
 // Bits [a, b) of a 32-bit word, with a and b clamped to [0, 32].
 __device__ __forceinline__ uint32_t range_bits(int a, int b)
 {
@@ -479,8 +448,7 @@ namespace bd {
 //  - S (128 fp32 columns at TMEM address ts) is read into registers.
 //  - On a PARTIAL tile, columns outside the row's visible intervals
 //    [sp.a0, sp.a1) U [sp.a2, sp.a3), or at or past key khi, become -inf
-//    (ks = first key of the tile).  With SKIP, 32-column words that no row of
-//    the warp sees also skip their max and exponentials.
+//    (ks = first key of the tile).
 //  - The running maximum m_used (log2 units) is raised lazily, only when the
 //    tile maximum exceeds it by more than 8; if any lane raises it and
 //    rescale_o is set, the warp waits for the previous PV (wait_prev_pv,
@@ -489,7 +457,7 @@ namespace bd {
 //  - P = 2^(s * sl2 - m_used) is written as bf16 over S, its sum added to l.
 // Returns false if wait_prev_pv failed.  The caller waits for the TMEM
 // stores and signals P.
-template <bool EMU, bool SKIP, typename WaitPV>
+template <bool EMU, typename WaitPV>
 __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool full,
                                              const Span &sp, int ks, int khi,
                                              float sl2, bool rescale_o,
@@ -506,49 +474,28 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
 #pragma unroll
     for (int c = 0; c < kTcN; ++c)
         s[c] = __uint_as_float(sr[c]);
-    uint32_t live = 0xFu;
     if (!full) {
         const int e = min(khi, ks + kTcN);
         const int lo0 = max(sp.a0, ks) - ks, hi0 = min(sp.a1, e) - ks;
         const int lo1 = max(sp.a2, ks) - ks, hi1 = min(sp.a3, e) - ks;
-        if (SKIP)
-            live = 0u;
 #pragma unroll
         for (int w = 0; w < kTcN / 32; ++w) {
             const uint32_t m = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
-            if (SKIP)
-                live |= (__any_sync(0xffffffffu, m != 0u) ? 1u : 0u) << w;
 #pragma unroll
             for (int c = 0; c < 32; ++c)
                 s[32 * w + c] = ((m >> c) & 1u) ? s[32 * w + c] : -INFINITY;
         }
     }
     float mc[8];
-    if (!SKIP || live == 0xFu) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        mc[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+    for (int c = 16; c < kTcN; c += 16)
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            mc[i] = fmaxf(s[i], s[8 + i]);
-#pragma unroll
-        for (int c = 16; c < kTcN; c += 16)
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
-    } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            mc[i] = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kTcN / 32; ++w) {
-            if ((live >> w) & 1u) {
-#pragma unroll
-                for (int c = 32 * w; c < 32 * w + 32; c += 16)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
-            }
-        }
-    }
+            mc[i] = fmax3(mc[i], s[c + i], s[c + 8 + i]);
     const float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]),
                            fmaxf(mc[6], mc[7]));
     const float mt = mx * sl2;
@@ -579,10 +526,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
     }
     const float nm = (m_used == -INFINITY) ? 0.f : -m_used;
     float rsum[4] = {0.f, 0.f, 0.f, 0.f};
-    if (!SKIP || live == 0xFu)
-        softmax_p_tile<EMU>(s, sl2, nm, ts, rsum);
-    else
-        softmax_p_tile_live(s, sl2, nm, ts, rsum, live);
+    softmax_p_tile<EMU>(s, sl2, nm, ts, rsum);
     l += (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
     return true;
 }

@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 tc_fence_after();
                 const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
                 const long long jp = jg - 1;
-                ok = softmax_tile<kEmuExp2, false>(
+                ok = softmax_tile<kEmuExp2>(
                     t_s + lane_off, t_o + lane_off, full, sp, ks, khi, sl2, jj >= 1, m_used, l,
                     [&] {
                         return mbar_wait(bar_odone(x, (int)(jp & 1)), (uint32_t)((jp >> 1) & 1),

@@ -594,7 +594,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 // the FMA-pipe exponential relieves the special-function
                 // unit where the softmax paces the tensor pipe (forward); the
                 // HBM-bound decode measured faster without it
-                ok = softmax_tile<KIND == 0 && kEmuExp2, false>(
+                ok = softmax_tile<KIND == 0 && kEmuExp2>(
                     t_s0 + (uint32_t)sb * 128 + lane_off, t_o + lane_off, full, sp, ks, khi, sl2,
                     jj >= 1, m_used, l, [&] {
                         return mbar_wait(bar_odone0 + 8 * (jp & 1), (uint32_t)((jp >> 1) & 1),
