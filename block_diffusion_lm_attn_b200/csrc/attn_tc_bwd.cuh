@@ -144,7 +144,7 @@ __device__ __forceinline__ void kv_step(const KvItem &it, int s, int &qhead,
 }
 
 // shared memory of the dK/dV kernel
-constexpr int kKvStages = 3;
+constexpr int kKvStages = 4;
 constexpr int kSubBytes = kBwdSub * kTcD * 2;              // 16 KB
 constexpr int kKvSmemK = 0;                                // K tile
 constexpr int kKvSmemV = kKvSmemK + kTileBytes;            // V tile
@@ -188,15 +188,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t bar0 = base + kKvSmemBar;
     const uint32_t bar_kvfull = bar0;        // K and V of the item landed
     const uint32_t bar_kvfree = bar0 + 8;    // every product of the item read K, V
-    auto bar_full = [&](int s) { return bar0 + 16 + 8 * s; };  // stage landed
-    auto bar_empty = [&](int s) { return bar0 + 40 + 8 * s; }; // stage read
-    auto bar_sfull = [&](int x) { return bar0 + 64 + 8 * x; }; // S^T, dP^T ready
-    auto bar_pfull = [&](int x) { return bar0 + 80 + 8 * x; }; // P^T, dS^T written
-    const uint32_t bar_odone = bar0 + 96;  // the item's last dV, dK retired
-    const uint32_t bar_ofree = bar0 + 104; // dV, dK read out
-    const uint32_t bar_final = bar0 + 112;
-    const uint32_t bar_ifull0 = bar0 + 120;  // 4: work item published
-    const uint32_t bar_iempty0 = bar0 + 152; // 4: work item read by all roles
+    auto bar_full = [&](int s) { return bar0 + 16 + 8 * s; };                  // stage landed
+    auto bar_empty = [&](int s) { return bar0 + 16 + 8 * kKvStages + 8 * s; }; // stage read
+    const uint32_t bar1 = bar0 + 16 + 16 * kKvStages;
+    auto bar_sfull = [&](int x) { return bar1 + 8 * x; };      // S^T, dP^T ready
+    auto bar_pfull = [&](int x) { return bar1 + 16 + 8 * x; }; // P^T, dS^T written
+    const uint32_t bar_odone = bar1 + 32;  // the item's last dV, dK retired
+    const uint32_t bar_ofree = bar1 + 40;  // dV, dK read out
+    const uint32_t bar_final = bar1 + 48;
+    const uint32_t bar_ifull0 = bar1 + 56;  // 4: work item published
+    const uint32_t bar_iempty0 = bar1 + 88; // 4: work item read by all roles
+    static_assert(16 + 16 * kKvStages + 120 <= 256, "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 256);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 384);
     volatile uint32_t *tmem_slot =
