@@ -72,6 +72,20 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// 4-byte global -> shared asynchronous copy; src_bytes = 0 writes zero.
+__device__ __forceinline__ void cp_async4(uint32_t dst, const float *src, int src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+// One arrival on `bar` once every cp.async this thread issued so far has
+// landed (counted among the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Query rows that see key position c (the transpose of fwd_span):
 //   noisy key of block k : noisy rows [k b, k b + b)
@@ -209,7 +223,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_kvfull, 1);
         mbar_init(bar_kvfree, 1);
         for (int s = 0; s < kKvStages; ++s) {
-            mbar_init(bar_full(s), 2); // expect_tx arrival + lse2/D arrival
+            mbar_init(bar_full(s), 1 + 32); // expect_tx arrival + one per producer lane
             mbar_init(bar_empty(s), 1);
         }
         for (int x = 0; x < 2; ++x) {
@@ -321,21 +335,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 bar_full(st));
                     iss = g + 1;
                 }
-                // lse2 and D of the 64 rows; rows outside the range get
-                // lse2 = +inf (P = 0)
+                // lse2 and D of the 64 rows, copied asynchronously (so that
+                // this warp goes on to the next stage at once); each lane's
+                // copies arrive on the stage barrier when they land.  Rows
+                // outside the range read as 0: the compute warps mask them
+                // (a step with such rows is never FULL).
                 const int hi = rg == 0 ? it.hi0 : it.hi1;
-                float *sl = reinterpret_cast<float *>(sbase + kKvSmemRows + st * kKvRowsBytes);
+                const uint32_t sl = base + kKvSmemRows + (uint32_t)st * kKvRowsBytes;
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
                     const int c = lane + 32 * u;
                     const long long row = (long long)qhead * 2 * p.L + qs + c;
                     const bool v = qs + c < hi && row < nrows_all;
-                    sl[c] = v ? p.lse2[row] : INFINITY;
-                    sl[kBwdSub + c] = v ? p.D[row] : 0.f;
+                    const long long r0 = v ? row : 0;
+                    cp_async4(sl + 4 * c, p.lse2 + r0, v ? 4 : 0);
+                    cp_async4(sl + 4 * (kBwdSub + c), p.D + r0, v ? 4 : 0);
                 }
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bar_full(st));
+                cp_async_arrive_noinc(bar_full(st));
             }
         }
         if (lane == 0) {
