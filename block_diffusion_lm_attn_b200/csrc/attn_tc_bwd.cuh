@@ -597,8 +597,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 constexpr int kDqSmemQ = 0;                          // Q tile
 constexpr int kDqSmemDO = kDqSmemQ + kTileBytes;     // dO tile
-constexpr int kDqSmemRing = kDqSmemDO + kTileBytes;  // 2 stages of K, V
-constexpr int kDqSmemBar = kDqSmemRing + 2 * 2 * kTileBytes;
+// K and V sit in rings of their own: V(t) is free once dP(t) has run, K(t)
+// only after dQ += dS(t) K(t), one tile later, so K gets the deeper ring.
+constexpr int kDqKStages = 3;
+constexpr int kDqVStages = 2;
+constexpr int kDqSmemK = kDqSmemDO + kTileBytes;               // K stages
+constexpr int kDqSmemV = kDqSmemK + kDqKStages * kTileBytes;  // V stages
+constexpr int kDqSmemBar = kDqSmemV + kDqVStages * kTileBytes;
 constexpr int kDqSmemBytes = kDqSmemBar + 512 + 1024;
 static_assert(kDqSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
@@ -622,17 +627,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t bar0 = base + kDqSmemBar;
     const uint32_t bar_qfull = bar0;      // Q and dO landed
     const uint32_t bar_qfree = bar0 + 8;  // every S, dP of the item retired
-    auto bar_kvfull = [&](int s) { return bar0 + 16 + 8 * s; };
-    auto bar_kvempty = [&](int s) { return bar0 + 32 + 8 * s; };
-    const uint32_t bar_sfull = bar0 + 48;  // S, dP ready
-    const uint32_t bar_sfree = bar0 + 56;  // S, dP read into registers
-    auto bar_dsfull = [&](int x) { return bar0 + 64 + 8 * x; };
-    auto bar_dsfree = [&](int x) { return bar0 + 80 + 8 * x; };
-    const uint32_t bar_qdone = bar0 + 96;  // the item's last dQ retired
-    const uint32_t bar_dqfree = bar0 + 104; // dQ read out
-    const uint32_t bar_final = bar0 + 112;
-    const uint32_t bar_ifull0 = bar0 + 120;
-    const uint32_t bar_iempty0 = bar0 + 152;
+    const uint32_t bar_sfull = bar0 + 16;  // S, dP ready
+    const uint32_t bar_sfree = bar0 + 24;  // S, dP read into registers
+    auto bar_dsfull = [&](int x) { return bar0 + 32 + 8 * x; };
+    auto bar_dsfree = [&](int x) { return bar0 + 48 + 8 * x; };
+    const uint32_t bar_qdone = bar0 + 64;  // the item's last dQ retired
+    const uint32_t bar_dqfree = bar0 + 72; // dQ read out
+    const uint32_t bar_final = bar0 + 80;
+    const uint32_t bar_ifull0 = bar0 + 88;
+    const uint32_t bar_iempty0 = bar0 + 120;
+    auto bar_kfull = [&](int s) { return bar0 + 152 + 8 * s; };
+    auto bar_kempty = [&](int s) { return bar0 + 152 + 8 * kDqKStages + 8 * s; };
+    auto bar_vfull = [&](int s) { return bar0 + 152 + 16 * kDqKStages + 8 * s; };
+    auto bar_vempty = [&](int s) { return bar0 + 152 + 16 * kDqKStages + 8 * kDqVStages + 8 * s; };
+    static_assert(152 + 16 * kDqKStages + 16 * kDqVStages <= 256, "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 256);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 384);
     volatile uint32_t *tmem_slot =
@@ -643,10 +651,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_qfull, 1);
         mbar_init(bar_qfree, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_kvfull(s), 1);
-            mbar_init(bar_kvempty(s), 1);
             mbar_init(bar_dsfull(s), 8); // one arrival per compute warp
             mbar_init(bar_dsfree(s), 1);
+        }
+        for (int s = 0; s < kDqKStages; ++s) {
+            mbar_init(bar_kfull(s), 1);
+            mbar_init(bar_kempty(s), 1);
+        }
+        for (int s = 0; s < kDqVStages; ++s) {
+            mbar_init(bar_vfull(s), 1);
+            mbar_init(bar_vempty(s), 1);
         }
         mbar_init(bar_sfull, 1);
         mbar_init(bar_sfree, 8);
@@ -712,7 +726,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int si = 0;
-            long long g = 0, iss = 0;
+            long long g = 0, issk = 0, issv = 0;
             while (ok && next_item(si, true, ok)) {
                 if (si >= 1 && !(ok = mbar_wait(bar_qfree, (uint32_t)((si - 1) & 1), abort_flag)))
                     break;
@@ -724,19 +738,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                             bar_qfull);
                 ++si;
                 for (int t = 0; t < sg.nt; ++t, ++g) {
-                    const int s = (int)(g & 1);
-                    if (g >= 2 && !(ok = mbar_wait(bar_kvempty(s), (uint32_t)(((g - 2) >> 1) & 1),
-                                                   abort_flag)))
-                        break;
                     const int ks = key_start(t);
-                    const uint32_t kb = base + kDqSmemRing + (uint32_t)s * 2 * kTileBytes;
-                    mbar_expect_tx(bar_kvfull(s), 2 * kTileBytes);
-                    tma_load_3d(kb, &tm_k, 0, ks, sg.kvhead, bar_kvfull(s));
-                    tma_load_3d(kb + kHalfTileBytes, &tm_k, 64, ks, sg.kvhead, bar_kvfull(s));
-                    tma_load_3d(kb + kTileBytes, &tm_v, 0, ks, sg.kvhead, bar_kvfull(s));
-                    tma_load_3d(kb + kTileBytes + kHalfTileBytes, &tm_v, 64, ks, sg.kvhead,
-                                bar_kvfull(s));
-                    iss = g + 1;
+                    const int sk = (int)(g % kDqKStages), sv = (int)(g % kDqVStages);
+                    if (g >= kDqKStages &&
+                        !(ok = mbar_wait(bar_kempty(sk), (uint32_t)(((g / kDqKStages) - 1) & 1),
+                                         abort_flag)))
+                        break;
+                    const uint32_t kb = base + kDqSmemK + (uint32_t)sk * kTileBytes;
+                    mbar_expect_tx(bar_kfull(sk), kTileBytes);
+                    tma_load_3d(kb, &tm_k, 0, ks, sg.kvhead, bar_kfull(sk));
+                    tma_load_3d(kb + kHalfTileBytes, &tm_k, 64, ks, sg.kvhead, bar_kfull(sk));
+                    issk = g + 1;
+                    if (g >= kDqVStages &&
+                        !(ok = mbar_wait(bar_vempty(sv), (uint32_t)(((g / kDqVStages) - 1) & 1),
+                                         abort_flag)))
+                        break;
+                    const uint32_t vb = base + kDqSmemV + (uint32_t)sv * kTileBytes;
+                    mbar_expect_tx(bar_vfull(sv), kTileBytes);
+                    tma_load_3d(vb, &tm_v, 0, ks, sg.kvhead, bar_vfull(sv));
+                    tma_load_3d(vb + kHalfTileBytes, &tm_v, 64, ks, sg.kvhead, bar_vfull(sv));
+                    issv = g + 1;
                 }
             }
             sched_finish(p.sched_slot);
@@ -746,8 +767,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             };
             if (si >= 1)
                 drain(bar_qfull, (uint32_t)((si - 1) & 1));
-            for (long long x = iss > 2 ? iss - 2 : 0; x < iss; ++x)
-                drain(bar_kvfull((int)(x & 1)), (uint32_t)((x >> 1) & 1));
+            for (long long x = issk > kDqKStages ? issk - kDqKStages : 0; x < issk; ++x)
+                drain(bar_kfull((int)(x % kDqKStages)), (uint32_t)((x / kDqKStages) & 1));
+            for (long long x = issv > kDqVStages ? issv - kDqVStages : 0; x < issv; ++x)
+                drain(bar_vfull((int)(x % kDqVStages)), (uint32_t)((x / kDqVStages) & 1));
         }
     } else if (warp == kBwdMmaWarp) {
         // ---------------------------------------------------- MMA issuer
@@ -758,8 +781,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool ok = true;
             int si = 0;
             long long j = 0; // running key-tile counter
-            auto issue_sdp = [&](long long jg) {
-                const uint32_t kb = base + kDqSmemRing + (uint32_t)(jg & 1) * 2 * kTileBytes;
+            // S = Q K^T once K(jg) has landed, dP = dO V^T once V(jg) has;
+            // V's stage is free again as soon as dP has run
+            auto issue_sdp = [&](long long jg) -> bool {
+                const int sk = (int)(jg % kDqKStages), sv = (int)(jg % kDqVStages);
+                if (!mbar_wait_warp(bar_kfull(sk), (uint32_t)((jg / kDqKStages) & 1), abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t kb = base + kDqSmemK + (uint32_t)sk * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
@@ -767,17 +796,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u,
                                 ld);
                 }
+                if (!mbar_wait_warp(bar_vfull(sv), (uint32_t)((jg / kDqVStages) & 1), abort_flag))
+                    return false;
+                tc_fence_after();
+                const uint32_t vb = base + kDqSmemV + (uint32_t)sv * kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                     tc_mma_ss_p(t_dp, smem_desc_sw128(base + kDqSmemDO + off, 16, 1024),
-                                smem_desc_sw128(kb + kTileBytes + off, 16, 1024), idesc_s,
+                                smem_desc_sw128(vb + off, 16, 1024), idesc_s,
                                 kk > 0 ? 1u : 0u, ld);
                 }
                 tc_commit_p(bar_sfull, ld);
+                tc_commit_p(bar_vempty(sv), ld);
+                return true;
             };
             auto issue_dq = [&](long long jg, bool first) {
-                const uint32_t kb = base + kDqSmemRing + (uint32_t)(jg & 1) * 2 * kTileBytes;
+                const uint32_t kb = base + kDqSmemK + (uint32_t)(jg % kDqKStages) * kTileBytes;
                 const int x = (int)(jg & 1);
 #pragma unroll
                 for (int kk = 0; kk < kTcN / 16; ++kk) {
@@ -786,7 +821,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 ld);
                 }
                 tc_commit_p(bar_dsfree(x), ld);
-                tc_commit_p(bar_kvempty(x), ld);
+                tc_commit_p(bar_kempty((int)(jg % kDqKStages)), ld);
             };
             for (;;) {
                 const bool got = next_item(si, false, ok, lane == 0);
@@ -798,15 +833,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int t = 0; t <= sg.nt && ok; ++t) {
                     const long long jg = j + t;
                     if (t < sg.nt) {
-                        if (!(ok = mbar_wait_warp(bar_kvfull((int)(jg & 1)),
-                                                  (uint32_t)((jg >> 1) & 1), abort_flag)))
-                            break;
                         // S, dP of the previous tile are in registers
                         if (jg >= 1 && !(ok = mbar_wait_warp(bar_sfree, (uint32_t)((jg - 1) & 1),
                                                              abort_flag)))
                             break;
-                        tc_fence_after();
-                        issue_sdp(jg);
+                        if (!(ok = issue_sdp(jg)))
+                            break;
                         if (t == sg.nt - 1)
                             tc_commit_p(bar_qfree, ld);
                     }
