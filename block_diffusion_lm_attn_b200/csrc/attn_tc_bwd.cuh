@@ -86,6 +86,45 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar)
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// Stores a warp's 32 rows of 64 bf16 each, held one row per lane (w = the
+// row's 32 packed words, lane = row), to row0 + r * stride for r < nvalid.
+// Rows written one per lane would make every 16-byte store touch 32
+// different lines; instead three xor-shuffle stages transpose the 8 x 8
+// grid of 16-byte chunks within each group of eight lanes, after which lane
+// 8a + u holds chunk u of rows 8a .. 8a + 7, and each of the eight stores
+// writes four whole 128-byte row pieces.
+__device__ __forceinline__ void warp_store_rows64(uint32_t (&w)[32], bf16 *row0, size_t stride,
+                                                  int nvalid, int lane)
+{
+    const int u = lane & 7;
+#pragma unroll
+    for (int m = 4; m >= 1; m >>= 1) {
+        const bool hi = (u & m) != 0;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            if (c & m)
+                continue;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t send = hi ? w[4 * c + e] : w[4 * (c | m) + e];
+                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+                if (hi)
+                    w[4 * c + e] = recv;
+                else
+                    w[4 * (c | m) + e] = recv;
+            }
+        }
+    }
+    const int a = lane >> 3;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int r = 8 * a + k;
+        if (r < nvalid)
+            reinterpret_cast<uint4 *>(row0 + (size_t)r * stride)[u] =
+                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Query rows that see key position c (the transpose of fwd_span):
 //   noisy key of block k : noisy rows [k b, k b + b)
@@ -550,30 +589,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
             // epilogue: dV and scale * dK, bf16; this thread's row, columns
             // 64 hc .. 64 hc + 63
-            const bool valid = row < it.nkeys;
-            const size_t grow = (size_t)it.kvhead * 2 * p.L + it.krow0 + row;
+            const size_t grow0 = (size_t)it.kvhead * 2 * p.L + it.krow0 + wq * 32;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {
                 const uint32_t tb = (which == 0 ? t_dv : t_dk) + lane_off + 64 * hc;
                 const float mul = which == 0 ? 1.f : p.scale;
-                bf16 *dst = (which == 0 ? p.dv : p.dk) + grow * kTcD + 64 * hc;
+                uint32_t o[64], w[32];
+                tmem_ld32(tb, o);
+                tmem_ld32(tb + 32, o + 32);
+                tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < 2; ++q4) {
-                    uint32_t o[32];
-                    tmem_ld32(tb + q4 * 32, o);
-                    tmem_wait_ld();
-                    if (valid) {
-#pragma unroll
-                        for (int i = 0; i < 32; i += 8) {
-                            uint4 v4;
-                            v4.x = pack_bf16x2(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul);
-                            v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * mul, __uint_as_float(o[i + 3]) * mul);
-                            v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * mul, __uint_as_float(o[i + 5]) * mul);
-                            v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * mul, __uint_as_float(o[i + 7]) * mul);
-                            reinterpret_cast<uint4 *>(dst)[q4 * 4 + i / 8] = v4;
-                        }
-                    }
-                }
+                for (int i = 0; i < 32; ++i)
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * mul,
+                                       __uint_as_float(o[2 * i + 1]) * mul);
+                warp_store_rows64(w, (which == 0 ? p.dv : p.dk) + grow0 * kTcD + 64 * hc, kTcD,
+                                  it.nkeys - wq * 32, lane);
             }
             tc_fence_before();
             __syncwarp();
@@ -957,24 +987,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            // this thread's row, dQ columns 64 hc .. 64 hc + 63
-#pragma unroll
-            for (int q4 = 0; q4 < 2; ++q4) {
-                uint32_t o[32];
-                tmem_ld32(t_dq + lane_off + 64 * hc + q4 * 32, o);
+            // the warp's 32 rows, dQ columns 64 hc .. 64 hc + 63
+            {
+                uint32_t o[64], w[32];
+                tmem_ld32(t_dq + lane_off + 64 * hc, o);
+                tmem_ld32(t_dq + lane_off + 64 * hc + 32, o + 32);
                 tmem_wait_ld();
-                if (valid) {
-                    const float mul = p.scale;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v4;
-                        v4.x = pack_bf16x2(__uint_as_float(o[i]) * mul, __uint_as_float(o[i + 1]) * mul);
-                        v4.y = pack_bf16x2(__uint_as_float(o[i + 2]) * mul, __uint_as_float(o[i + 3]) * mul);
-                        v4.z = pack_bf16x2(__uint_as_float(o[i + 4]) * mul, __uint_as_float(o[i + 5]) * mul);
-                        v4.w = pack_bf16x2(__uint_as_float(o[i + 6]) * mul, __uint_as_float(o[i + 7]) * mul);
-                        reinterpret_cast<uint4 *>(p.dq + grow * kTcD + 64 * hc)[q4 * 4 + i / 8] = v4;
-                    }
-                }
+                for (int i = 0; i < 32; ++i)
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * p.scale,
+                                       __uint_as_float(o[2 * i + 1]) * p.scale);
+                warp_store_rows64(w, p.dq + (grow - lane) * kTcD + 64 * hc, kTcD,
+                                  sg.nrows - wq * 32, lane);
             }
             tc_fence_before();
             __syncwarp();
