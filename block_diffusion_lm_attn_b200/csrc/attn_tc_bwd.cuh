@@ -44,31 +44,48 @@ struct BParams {
 };
 
 // ---------------------------------------------------------------------------
-// D and lse * log2(e), one warp per query row of 128 values.
+// D and lse * log2(e) per query row of 128 values.  A half-warp reduces one
+// row from 16-byte loads; each warp takes four rows and issues all its loads
+// before any reduction, so enough bytes are in flight to stream at HBM rate.
+constexpr int kPrepRowsPerBlock = 32; // 8 warps x 4 rows
 
 __global__ void __launch_bounds__(256)
     bd_bwd_prep_kernel(const BParams p, long long rows)
 {
-    const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (r >= rows)
-        return;
-    const uint2 o = reinterpret_cast<const uint2 *>(p.out + r * kTcD)[lane];
-    const uint2 g = reinterpret_cast<const uint2 *>(p.dout + r * kTcD)[lane];
-    const uint32_t ow[2] = {o.x, o.y}, gw[2] = {g.x, g.y};
-    float acc = 0.f;
+    const int lane = threadIdx.x & 31, hw = lane >> 4, l16 = lane & 15;
+    const long long r0 = (long long)blockIdx.x * kPrepRowsPerBlock + (threadIdx.x >> 5) * 4;
+    uint4 o[2], g[2];
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        acc = fmaf(__uint_as_float(ow[t] << 16), __uint_as_float(gw[t] << 16), acc);
-        acc = fmaf(__uint_as_float(ow[t] & 0xffff0000u), __uint_as_float(gw[t] & 0xffff0000u), acc);
+    for (int i = 0; i < 2; ++i) {
+        const long long r = r0 + 2 * i + hw;
+        if (r < rows) {
+            o[i] = __ldg(reinterpret_cast<const uint4 *>(p.out + r * kTcD) + l16);
+            g[i] = __ldg(reinterpret_cast<const uint4 *>(p.dout + r * kTcD) + l16);
+        } else {
+            o[i] = make_uint4(0, 0, 0, 0);
+            g[i] = o[i];
+        }
     }
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1)
-        acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (lane == 0) {
-        p.D[r] = acc;
-        const float l = p.lse[r];
-        p.lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+    for (int i = 0; i < 2; ++i) {
+        const uint32_t ow[4] = {o[i].x, o[i].y, o[i].z, o[i].w};
+        const uint32_t gw[4] = {g[i].x, g[i].y, g[i].z, g[i].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            acc = fmaf(__uint_as_float(ow[t] << 16), __uint_as_float(gw[t] << 16), acc);
+            acc = fmaf(__uint_as_float(ow[t] & 0xffff0000u), __uint_as_float(gw[t] & 0xffff0000u),
+                       acc);
+        }
+#pragma unroll
+        for (int m = 8; m > 0; m >>= 1)
+            acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        const long long r = r0 + 2 * i + hw;
+        if (l16 == 0 && r < rows) {
+            p.D[r] = acc;
+            const float l = p.lse[r];
+            p.lse2[r] = (l == -INFINITY) ? INFINITY : l * kLog2e;
+        }
     }
 }
 

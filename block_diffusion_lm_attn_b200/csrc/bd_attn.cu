@@ -540,7 +540,8 @@ bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
         !make_map_rows(&mv, v, N, (uint64_t)B * Hkv, 128))
         return BD_ERR_CUDA;
 
-    bd::bd_bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(p, (long long)rows);
+    bd::bd_bwd_prep_kernel<<<(unsigned)((rows + bd::kPrepRowsPerBlock - 1) / bd::kPrepRowsPerBlock),
+                             256, 0, stream>>>(p, (long long)rows);
     if (cudaGetLastError() != cudaSuccess)
         return BD_ERR_CUDA;
 
