@@ -244,34 +244,154 @@ __device__ __forceinline__ void tc_commit_p(uint32_t bar, uint32_t leader)
                  : "memory");
 }
 
-// 32 lanes x 32 columns of 32-bit TMEM words -> 32 registers per thread
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
+// TMEM loads, shape 32x32b: thread i of the warp reads TMEM lane
+// 32 * (warp id mod 4) + i, consecutive 32-bit columns from the address's
+// column on; each is fused with its tcgen05.wait::ld in one statement.  The destination registers are defined
+// only once the loads have landed, so the compiler can neither read them
+// early nor spill them while a load is in flight; a separate load and wait
+// would be correct only if nothing between the two touched the registers,
+// which the compiler does not know.
+// 32 columns
+__device__ __forceinline__ void tmem_ld32_wait(uint32_t a0, uint32_t *r0)
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
-        "[%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
-          "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
-          "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
-          "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31"
+        "}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]),
+          "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]),
+          "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]),
+          "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]),
+          "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]),
+          "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]),
+          "=r"(r0[30]), "=r"(r0[31])
+        : "r"(a0)
+        : "memory");
 }
-// 32 lanes x 16 columns -> 16 registers per thread
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r)
+// two loads of 32 columns from a0 and a1
+__device__ __forceinline__ void tmem_ld32x2_wait(uint32_t a0, uint32_t a1, uint32_t *r0, uint32_t *r1)
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
-          "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
-          "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-          "=r"(r[15])
-        : "r"(taddr));
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31"
+        "}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63"
+        "}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]),
+          "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]),
+          "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]),
+          "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]),
+          "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]),
+          "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]),
+          "=r"(r0[30]), "=r"(r0[31]), "=r"(r1[0]), "=r"(r1[1]), "=r"(r1[2]),
+          "=r"(r1[3]), "=r"(r1[4]), "=r"(r1[5]), "=r"(r1[6]), "=r"(r1[7]),
+          "=r"(r1[8]), "=r"(r1[9]), "=r"(r1[10]), "=r"(r1[11]), "=r"(r1[12]),
+          "=r"(r1[13]), "=r"(r1[14]), "=r"(r1[15]), "=r"(r1[16]), "=r"(r1[17]),
+          "=r"(r1[18]), "=r"(r1[19]), "=r"(r1[20]), "=r"(r1[21]), "=r"(r1[22]),
+          "=r"(r1[23]), "=r"(r1[24]), "=r"(r1[25]), "=r"(r1[26]), "=r"(r1[27]),
+          "=r"(r1[28]), "=r"(r1[29]), "=r"(r1[30]), "=r"(r1[31])
+        : "r"(a0), "r"(a1)
+        : "memory");
+}
+// four loads of 32 columns from a0 .. a3
+__device__ __forceinline__ void tmem_ld32x4_wait(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t *r0, uint32_t *r1, uint32_t *r2, uint32_t *r3)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31"
+        "}, [%128];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63"
+        "}, [%129];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95"
+        "}, [%130];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+        "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+        "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127"
+        "}, [%131];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]),
+          "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]),
+          "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]),
+          "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]),
+          "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]),
+          "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]),
+          "=r"(r0[30]), "=r"(r0[31]), "=r"(r1[0]), "=r"(r1[1]), "=r"(r1[2]),
+          "=r"(r1[3]), "=r"(r1[4]), "=r"(r1[5]), "=r"(r1[6]), "=r"(r1[7]),
+          "=r"(r1[8]), "=r"(r1[9]), "=r"(r1[10]), "=r"(r1[11]), "=r"(r1[12]),
+          "=r"(r1[13]), "=r"(r1[14]), "=r"(r1[15]), "=r"(r1[16]), "=r"(r1[17]),
+          "=r"(r1[18]), "=r"(r1[19]), "=r"(r1[20]), "=r"(r1[21]), "=r"(r1[22]),
+          "=r"(r1[23]), "=r"(r1[24]), "=r"(r1[25]), "=r"(r1[26]), "=r"(r1[27]),
+          "=r"(r1[28]), "=r"(r1[29]), "=r"(r1[30]), "=r"(r1[31]), "=r"(r2[0]),
+          "=r"(r2[1]), "=r"(r2[2]), "=r"(r2[3]), "=r"(r2[4]), "=r"(r2[5]),
+          "=r"(r2[6]), "=r"(r2[7]), "=r"(r2[8]), "=r"(r2[9]), "=r"(r2[10]),
+          "=r"(r2[11]), "=r"(r2[12]), "=r"(r2[13]), "=r"(r2[14]), "=r"(r2[15]),
+          "=r"(r2[16]), "=r"(r2[17]), "=r"(r2[18]), "=r"(r2[19]), "=r"(r2[20]),
+          "=r"(r2[21]), "=r"(r2[22]), "=r"(r2[23]), "=r"(r2[24]), "=r"(r2[25]),
+          "=r"(r2[26]), "=r"(r2[27]), "=r"(r2[28]), "=r"(r2[29]), "=r"(r2[30]),
+          "=r"(r2[31]), "=r"(r3[0]), "=r"(r3[1]), "=r"(r3[2]), "=r"(r3[3]),
+          "=r"(r3[4]), "=r"(r3[5]), "=r"(r3[6]), "=r"(r3[7]), "=r"(r3[8]),
+          "=r"(r3[9]), "=r"(r3[10]), "=r"(r3[11]), "=r"(r3[12]), "=r"(r3[13]),
+          "=r"(r3[14]), "=r"(r3[15]), "=r"(r3[16]), "=r"(r3[17]), "=r"(r3[18]),
+          "=r"(r3[19]), "=r"(r3[20]), "=r"(r3[21]), "=r"(r3[22]), "=r"(r3[23]),
+          "=r"(r3[24]), "=r"(r3[25]), "=r"(r3[26]), "=r"(r3[27]), "=r"(r3[28]),
+          "=r"(r3[29]), "=r"(r3[30]), "=r"(r3[31])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
+        : "memory");
+}
+// 128 columns in one load
+__device__ __forceinline__ void tmem_ld128_wait(uint32_t a0, uint32_t *r0)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+        "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+        "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+        "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127"
+        "}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]),
+          "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]),
+          "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]),
+          "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]),
+          "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]),
+          "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]),
+          "=r"(r0[30]), "=r"(r0[31]), "=r"(r0[32]), "=r"(r0[33]), "=r"(r0[34]),
+          "=r"(r0[35]), "=r"(r0[36]), "=r"(r0[37]), "=r"(r0[38]), "=r"(r0[39]),
+          "=r"(r0[40]), "=r"(r0[41]), "=r"(r0[42]), "=r"(r0[43]), "=r"(r0[44]),
+          "=r"(r0[45]), "=r"(r0[46]), "=r"(r0[47]), "=r"(r0[48]), "=r"(r0[49]),
+          "=r"(r0[50]), "=r"(r0[51]), "=r"(r0[52]), "=r"(r0[53]), "=r"(r0[54]),
+          "=r"(r0[55]), "=r"(r0[56]), "=r"(r0[57]), "=r"(r0[58]), "=r"(r0[59]),
+          "=r"(r0[60]), "=r"(r0[61]), "=r"(r0[62]), "=r"(r0[63]), "=r"(r0[64]),
+          "=r"(r0[65]), "=r"(r0[66]), "=r"(r0[67]), "=r"(r0[68]), "=r"(r0[69]),
+          "=r"(r0[70]), "=r"(r0[71]), "=r"(r0[72]), "=r"(r0[73]), "=r"(r0[74]),
+          "=r"(r0[75]), "=r"(r0[76]), "=r"(r0[77]), "=r"(r0[78]), "=r"(r0[79]),
+          "=r"(r0[80]), "=r"(r0[81]), "=r"(r0[82]), "=r"(r0[83]), "=r"(r0[84]),
+          "=r"(r0[85]), "=r"(r0[86]), "=r"(r0[87]), "=r"(r0[88]), "=r"(r0[89]),
+          "=r"(r0[90]), "=r"(r0[91]), "=r"(r0[92]), "=r"(r0[93]), "=r"(r0[94]),
+          "=r"(r0[95]), "=r"(r0[96]), "=r"(r0[97]), "=r"(r0[98]), "=r"(r0[99]),
+          "=r"(r0[100]), "=r"(r0[101]), "=r"(r0[102]), "=r"(r0[103]), "=r"(r0[104]),
+          "=r"(r0[105]), "=r"(r0[106]), "=r"(r0[107]), "=r"(r0[108]), "=r"(r0[109]),
+          "=r"(r0[110]), "=r"(r0[111]), "=r"(r0[112]), "=r"(r0[113]), "=r"(r0[114]),
+          "=r"(r0[115]), "=r"(r0[116]), "=r"(r0[117]), "=r"(r0[118]), "=r"(r0[119]),
+          "=r"(r0[120]), "=r"(r0[121]), "=r"(r0[122]), "=r"(r0[123]), "=r"(r0[124]),
+          "=r"(r0[125]), "=r"(r0[126]), "=r"(r0[127])
+        : "r"(a0)
+        : "memory");
 }
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
 {
@@ -298,10 +418,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r)
         "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
         "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld()
-{
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_wait_st()
 {
@@ -465,11 +581,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
                                              WaitPV wait_prev_pv)
 {
     uint32_t sr[kTcN];
-    tmem_ld32(ts + 0, sr + 0);
-    tmem_ld32(ts + 32, sr + 32);
-    tmem_ld32(ts + 64, sr + 64);
-    tmem_ld32(ts + 96, sr + 96);
-    tmem_wait_ld();
+    tmem_ld32x4_wait(ts, ts + 32, ts + 64, ts + 96, sr, sr + 32, sr + 64, sr + 96);
     float s[kTcN];
 #pragma unroll
     for (int c = 0; c < kTcN; ++c)
@@ -516,8 +628,7 @@ __device__ __forceinline__ bool softmax_tile(uint32_t ts, uint32_t t_o, bool ful
 #pragma unroll
         for (int q4 = 0; q4 < kTcD / 32; ++q4) {
             uint32_t o[32];
-            tmem_ld32(t_o + q4 * 32, o);
-            tmem_wait_ld();
+            tmem_ld32_wait(t_o + q4 * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 o[i] = __float_as_uint(__uint_as_float(o[i]) * c);

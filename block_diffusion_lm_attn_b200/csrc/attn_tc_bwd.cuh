@@ -551,9 +551,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     break;
                 tc_fence_after();
                 uint32_t sr[32], dr[32];
-                tmem_ld32(t_st(x) + lane_off + 32 * hc, sr);
-                tmem_ld32(t_dp(x) + lane_off + 32 * hc, dr);
-                tmem_wait_ld();
+                tmem_ld32x2_wait(t_st(x) + lane_off + 32 * hc, t_dp(x) + lane_off + 32 * hc, sr, dr);
                 const float *sl = reinterpret_cast<const float *>(
                                       sbase + kKvSmemRows + st * kKvRowsBytes) + 32 * hc;
                 const int hi = rg == 0 ? it.hi0 : it.hi1;
@@ -612,9 +610,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t tb = (which == 0 ? t_dv : t_dk) + lane_off + 64 * hc;
                 const float mul = which == 0 ? 1.f : p.scale;
                 uint32_t o[64], w[32];
-                tmem_ld32(tb, o);
-                tmem_ld32(tb + 32, o + 32);
-                tmem_wait_ld();
+                tmem_ld32x2_wait(tb, tb + 32, o, o + 32);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * mul,
@@ -960,11 +956,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                 range_bits(lo1 - 32 * w, hi1 - 32 * w);
                 }
                 uint32_t sr[64], dr[64], pk[32];
-                tmem_ld32(t_s + lane_off + 64 * hc, sr);
-                tmem_ld32(t_s + lane_off + 64 * hc + 32, sr + 32);
-                tmem_ld32(t_dp + lane_off + 64 * hc, dr);
-                tmem_ld32(t_dp + lane_off + 64 * hc + 32, dr + 32);
-                tmem_wait_ld();
+                tmem_ld32x4_wait(t_s + lane_off + 64 * hc, t_s + lane_off + 64 * hc + 32,
+                                 t_dp + lane_off + 64 * hc, t_dp + lane_off + 64 * hc + 32, sr,
+                                 sr + 32, dr, dr + 32);
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0)
@@ -1007,9 +1001,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             // the warp's 32 rows, dQ columns 64 hc .. 64 hc + 63
             {
                 uint32_t o[64], w[32];
-                tmem_ld32(t_dq + lane_off + 64 * hc, o);
-                tmem_ld32(t_dq + lane_off + 64 * hc + 32, o + 32);
-                tmem_wait_ld();
+                tmem_ld32x2_wait(t_dq + lane_off + 64 * hc, t_dq + lane_off + 64 * hc + 32, o,
+                                 o + 32);
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * p.scale,

@@ -447,8 +447,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 for (int q = 0; q < 2; ++q) {
                     const int q4 = 2 * h + q;
                     uint32_t o[32];
-                    tmem_ld32(t_o + lane_off + q4 * 32, o);
-                    tmem_wait_ld();
+                    tmem_ld32_wait(t_o + lane_off + q4 * 32, o);
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         const uint32_t cch = (uint32_t)(q * 4 + i / 8);

@@ -641,8 +641,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if (q4 * 32 >= DH) // O columns past the head dim are not output
                     break;
                 uint32_t o[32];
-                tmem_ld32(t_o + lane_off + q4 * 32, o);
-                tmem_wait_ld();
+                tmem_ld32_wait(t_o + lane_off + q4 * 32, o);
                 if (kStage) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
