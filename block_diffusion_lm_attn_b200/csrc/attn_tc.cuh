@@ -349,50 +349,6 @@ __device__ __forceinline__ void tmem_ld32x4_wait(uint32_t a0, uint32_t a1, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
         : "memory");
 }
-// 128 columns in one load
-__device__ __forceinline__ void tmem_ld128_wait(uint32_t a0, uint32_t *r0)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
-        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
-        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
-        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
-        "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
-        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
-        "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
-        "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127"
-        "}, [%128];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]),
-          "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]),
-          "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]),
-          "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]),
-          "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]),
-          "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]),
-          "=r"(r0[30]), "=r"(r0[31]), "=r"(r0[32]), "=r"(r0[33]), "=r"(r0[34]),
-          "=r"(r0[35]), "=r"(r0[36]), "=r"(r0[37]), "=r"(r0[38]), "=r"(r0[39]),
-          "=r"(r0[40]), "=r"(r0[41]), "=r"(r0[42]), "=r"(r0[43]), "=r"(r0[44]),
-          "=r"(r0[45]), "=r"(r0[46]), "=r"(r0[47]), "=r"(r0[48]), "=r"(r0[49]),
-          "=r"(r0[50]), "=r"(r0[51]), "=r"(r0[52]), "=r"(r0[53]), "=r"(r0[54]),
-          "=r"(r0[55]), "=r"(r0[56]), "=r"(r0[57]), "=r"(r0[58]), "=r"(r0[59]),
-          "=r"(r0[60]), "=r"(r0[61]), "=r"(r0[62]), "=r"(r0[63]), "=r"(r0[64]),
-          "=r"(r0[65]), "=r"(r0[66]), "=r"(r0[67]), "=r"(r0[68]), "=r"(r0[69]),
-          "=r"(r0[70]), "=r"(r0[71]), "=r"(r0[72]), "=r"(r0[73]), "=r"(r0[74]),
-          "=r"(r0[75]), "=r"(r0[76]), "=r"(r0[77]), "=r"(r0[78]), "=r"(r0[79]),
-          "=r"(r0[80]), "=r"(r0[81]), "=r"(r0[82]), "=r"(r0[83]), "=r"(r0[84]),
-          "=r"(r0[85]), "=r"(r0[86]), "=r"(r0[87]), "=r"(r0[88]), "=r"(r0[89]),
-          "=r"(r0[90]), "=r"(r0[91]), "=r"(r0[92]), "=r"(r0[93]), "=r"(r0[94]),
-          "=r"(r0[95]), "=r"(r0[96]), "=r"(r0[97]), "=r"(r0[98]), "=r"(r0[99]),
-          "=r"(r0[100]), "=r"(r0[101]), "=r"(r0[102]), "=r"(r0[103]), "=r"(r0[104]),
-          "=r"(r0[105]), "=r"(r0[106]), "=r"(r0[107]), "=r"(r0[108]), "=r"(r0[109]),
-          "=r"(r0[110]), "=r"(r0[111]), "=r"(r0[112]), "=r"(r0[113]), "=r"(r0[114]),
-          "=r"(r0[115]), "=r"(r0[116]), "=r"(r0[117]), "=r"(r0[118]), "=r"(r0[119]),
-          "=r"(r0[120]), "=r"(r0[121]), "=r"(r0[122]), "=r"(r0[123]), "=r"(r0[124]),
-          "=r"(r0[125]), "=r"(r0[126]), "=r"(r0[127])
-        : "r"(a0)
-        : "memory");
-}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
 {
     asm volatile(

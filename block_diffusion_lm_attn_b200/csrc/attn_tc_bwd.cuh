@@ -17,7 +17,7 @@
 //   bd_bwd_prep_kernel   D_i and lse_i * log2(e) per query row (HBM-bound);
 //   bd_bwd_dkdv_kernel   one persistent CTA per SM; a work item is one
 //                        128-key tile of one kv-head; it walks the q-heads of
-//                        the group and, in 64-row steps, the query rows that
+//                        the group and, in 128-row steps, the query rows that
 //                        see the tile (the transpose of the forward's key
 //                        ranges), accumulating dV and dK in tensor memory;
 //   bd_bwd_dq_kernel     one persistent CTA per SM; a work item is one
@@ -159,7 +159,7 @@ __device__ __forceinline__ Span key_span(int L, int b, int c)
     return s;
 }
 
-constexpr int kBwdSub = 64; // query rows per step of the dK/dV kernel
+constexpr int kBwdSub = 128; // query rows per step of the dK/dV kernel
 
 // Work item of the dK/dV kernel: (batch, kv-head) = w / R, rank r = w % R:
 // clean key tiles first (they are seen by the most query rows), idx
@@ -170,7 +170,7 @@ struct KvItem {
     int krow0, nkeys; // first key row (of 2L), valid keys (<= 128)
     int lo0, hi0, lo1, hi1;     // query ranges
     int flo0, fhi0, flo1, fhi1; // queries every key of the tile sees
-    int n0, n1;       // 64-row steps of range 0 / range 1 per q-head
+    int n0, n1;       // steps of range 0 / range 1 per q-head
     int nt;           // steps of the item (all q-heads)
 };
 
@@ -214,8 +214,8 @@ __device__ __forceinline__ void kv_step(const KvItem &it, int s, int &qhead,
 }
 
 // shared memory of the dK/dV kernel
-constexpr int kKvStages = 4;
-constexpr int kSubBytes = kBwdSub * kTcD * 2;              // 16 KB
+constexpr int kKvStages = 2;
+constexpr int kSubBytes = kBwdSub * kTcD * 2;              // one step of Q or dO: 32 KB
 constexpr int kKvSmemK = 0;                                // K tile
 constexpr int kKvSmemV = kKvSmemK + kTileBytes;            // V tile
 constexpr int kKvSmemRing = kKvSmemV + kTileBytes;         // stages: Q, dO
@@ -233,21 +233,24 @@ constexpr int kBwdThreads = 320;
 constexpr int kBwdProducerWarp = 8, kBwdMmaWarp = 9;
 
 // Roles: warps 0-7 compute P^T and dS^T (warp w: key rows of TMEM lane
-// quarter w & 3, half w >> 2 of each step's query columns) and write dK, dV
-// out; warp 8 loads (TMA for tiles, plain loads for the per-row lse2 and D)
-// and fetches work items; warp 9 issues the MMAs.
-// TMEM: dV [0,128), dK [128,256); two buffers x of S^T [256 + 128x, +64)
-// and dP^T [320 + 128x, +64); P^T (bf16) overwrites its S^T, dS^T its dP^T.
-// Per step s (64 query rows, buffer x = s & 1):
-//   S^T = K Q^T, dP^T = V dO^T into buffer x, then for step s - 1:
-//   dV += P^T dO, dK += dS^T Q from buffer x ^ 1 (tcgen05.mma from one
-//   thread execute in issue order, so buffer x is rewritten only after the
-//   products of step s - 2 that read it).
+// quarter w & 3, query columns 64 hc .. 64 hc + 63 of each step, hc = w >> 2)
+// and write dK, dV out; warp 8 loads (TMA for tiles, cp.async for the
+// per-row lse2 and D) and fetches work items; warp 9 issues the MMAs.
+// TMEM: dV [0,128), dK [128,256), S^T [256,384), dP^T [384,512); P^T (bf16)
+// overwrites the S^T columns of the warp that formed it, dS^T those of dP^T.
+// Every product has M = 128 keys and N = 128 (queries or head dim), the
+// full-rate shape.  Issue order, step s of 128 query rows:
+//   ... dV(s-1), S^T(s), dK(s-1), dP^T(s), dV(s), S^T(s+1), dK(s), ...
+// S^T(s+1) rewrites the columns P^T(s) sits in only after dV(s), which reads
+// them, was issued, and dP^T(s+1) those of dS^T(s) only after dK(s)
+// (tcgen05.mma from one thread execute in issue order).  The compute warps
+// form P^T(s) while dK(s-1) and dP^T(s) run, then dS^T(s) (from P^T(s) in
+// registers and dP^T(s)) while dV(s) and S^T(s+1) run.
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bd_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_q64,
-                       const __grid_constant__ CUtensorMap tm_do64,
+                       const __grid_constant__ CUtensorMap tm_qs,
+                       const __grid_constant__ CUtensorMap tm_dos,
                        const BParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -261,10 +264,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar_full = [&](int s) { return bar0 + 16 + 8 * s; };                  // stage landed
     auto bar_empty = [&](int s) { return bar0 + 16 + 8 * kKvStages + 8 * s; }; // stage read
     const uint32_t bar1 = bar0 + 16 + 16 * kKvStages;
-    auto bar_sfull = [&](int x) { return bar1 + 8 * x; };      // S^T, dP^T ready
-    auto bar_pfull = [&](int x) { return bar1 + 16 + 8 * x; }; // P^T, dS^T written
-    const uint32_t bar_odone = bar1 + 32;  // the item's last dV, dK retired
-    const uint32_t bar_ofree = bar1 + 40;  // dV, dK read out
+    const uint32_t bar_sdone = bar1;        // S^T ready
+    const uint32_t bar_dpdone = bar1 + 8;   // dP^T ready
+    const uint32_t bar_pready = bar1 + 16;  // P^T written
+    const uint32_t bar_dsready = bar1 + 24; // dS^T written
+    const uint32_t bar_odone = bar1 + 32;   // the item's last dV, dK retired
+    const uint32_t bar_ofree = bar1 + 40;   // dV, dK read out
     const uint32_t bar_final = bar1 + 48;
     const uint32_t bar_ifull0 = bar1 + 56;  // 4: work item published
     const uint32_t bar_iempty0 = bar1 + 88; // 4: work item read by all roles
@@ -282,10 +287,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(bar_full(s), 1 + 32); // expect_tx arrival + one per producer lane
             mbar_init(bar_empty(s), 1);
         }
-        for (int x = 0; x < 2; ++x) {
-            mbar_init(bar_sfull(x), 1);
-            mbar_init(bar_pfull(x), 8); // one arrival per compute warp
-        }
+        mbar_init(bar_sdone, 1);
+        mbar_init(bar_dpdone, 1);
+        mbar_init(bar_pready, 8); // one arrival per compute warp
+        mbar_init(bar_dsready, 8);
         mbar_init(bar_odone, 1);
         mbar_init(bar_ofree, 8);
         mbar_init(bar_final, 1);
@@ -306,9 +311,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_dv = tmem, t_dk = tmem + 128;
-    auto t_st = [&](int x) { return tmem + 256 + 128 * (uint32_t)x; };
-    auto t_dp = [&](int x) { return tmem + 320 + 128 * (uint32_t)x; };
+    const uint32_t t_dv = tmem, t_dk = tmem + 128, t_st = tmem + 256, t_dp = tmem + 384;
 
     KvItem it;
     auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
@@ -384,22 +387,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
                 if (lane == 0) {
                     mbar_expect_tx(bar_full(st), 2 * kSubBytes);
-                    tma_load_3d(sb, &tm_q64, 0, qs, qhead, bar_full(st));
-                    tma_load_3d(sb + kSubBytes / 2, &tm_q64, 64, qs, qhead, bar_full(st));
-                    tma_load_3d(sb + kSubBytes, &tm_do64, 0, qs, qhead, bar_full(st));
-                    tma_load_3d(sb + kSubBytes + kSubBytes / 2, &tm_do64, 64, qs, qhead,
+                    tma_load_3d(sb, &tm_qs, 0, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes / 2, &tm_qs, 64, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes, &tm_dos, 0, qs, qhead, bar_full(st));
+                    tma_load_3d(sb + kSubBytes + kSubBytes / 2, &tm_dos, 64, qs, qhead,
                                 bar_full(st));
                     iss = g + 1;
                 }
-                // lse2 and D of the 64 rows, copied asynchronously (so that
-                // this warp goes on to the next stage at once); each lane's
-                // copies arrive on the stage barrier when they land.  Rows
-                // outside the range read as 0: the compute warps mask them
-                // (a step with such rows is never FULL).
+                // lse2 and D of the step's rows, copied asynchronously (so
+                // that this warp goes on to the next stage at once); each
+                // lane's copies arrive on the stage barrier when they land.
+                // Rows outside the range read as 0: the compute warps mask
+                // them (a step with such rows is never FULL).
                 const int hi = rg == 0 ? it.hi0 : it.hi1;
                 const uint32_t sl = base + kKvSmemRows + (uint32_t)st * kKvRowsBytes;
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < kBwdSub / 32; ++u) {
                     const int c = lane + 32 * u;
                     const long long row = (long long)qhead * 2 * p.L + qs + c;
                     const bool v = qs + c < hi && row < nrows_all;
@@ -430,47 +433,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bool ok = true;
             int si = 0;
             long long g = 0;
-            auto issue_sdp = [&](long long gg) {
-                const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
-                const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
-#pragma unroll
-                for (int kk = 0; kk < kTcD / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
-                    tc_mma_ss_p(t_st(x), smem_desc_sw128(base + kKvSmemK + ao, 16, 1024),
-                                smem_desc_sw128(sb + bo, 16, 1024), idesc_s, kk > 0 ? 1u : 0u,
-                                ld);
-                }
-#pragma unroll
-                for (int kk = 0; kk < kTcD / 16; ++kk) {
-                    const uint32_t ao = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
-                    const uint32_t bo = (kk >> 2) * (kSubBytes / 2) + (kk & 3) * 32;
-                    tc_mma_ss_p(t_dp(x), smem_desc_sw128(base + kKvSmemV + ao, 16, 1024),
-                                smem_desc_sw128(sb + kSubBytes + bo, 16, 1024), idesc_s,
-                                kk > 0 ? 1u : 0u, ld);
-                }
-                tc_commit_p(bar_sfull(x), ld);
+            auto stage = [&](long long gg) {
+                return base + kKvSmemRing + (uint32_t)(gg % kKvStages) * kKvStageBytes;
             };
-            auto issue_grad = [&](long long gg, bool first) {
-                const int st = (int)(gg % kKvStages), x = (int)(gg & 1);
-                const uint32_t sb = base + kKvSmemRing + (uint32_t)st * kKvStageBytes;
-                // K-step kk covers queries 16 kk .. 16 kk + 15, packed by the
-                // compute warps of half kk / 2 at columns 32 (kk / 2) + 8 (kk % 2)
+            auto wait_stage = [&](long long gg) {
+                return mbar_wait_warp(bar_full((int)(gg % kKvStages)),
+                                      (uint32_t)((gg / kKvStages) & 1), abort_flag);
+            };
+            // S^T = K Q^T (A = operand a_tile, B = the stage's Q) or
+            // dP^T = V dO^T: M = 128 keys, N = 128 queries, 8 K-steps over d
+            auto issue_t = [&](uint32_t acc, uint32_t a_tile, uint32_t b_tile, uint32_t bar) {
 #pragma unroll
-                for (int kk = 0; kk < kBwdSub / 16; ++kk) {
-                    const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
-                    const uint64_t bdo = smem_desc_sw128(sb + kSubBytes + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts_p(t_dv, t_st(x) + acol, bdo, idesc_g, (!first || kk > 0) ? 1u : 0u,
+                for (int kk = 0; kk < kTcD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
+                    tc_mma_ss_p(acc, smem_desc_sw128(a_tile + off, 16, 1024),
+                                smem_desc_sw128(b_tile + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u,
                                 ld);
                 }
+                tc_commit_p(bar, ld);
+            };
+            // dV += P^T dO or dK += dS^T Q: A from TMEM (K-step kk = queries
+            // 16 kk .. 16 kk + 15, packed by the warps of half kk / 4 at
+            // columns 64 (kk / 4) + 8 (kk % 4)), B = dO or Q of the stage
+            auto issue_g = [&](uint32_t acc, uint32_t a_tm, uint32_t b_tile, bool first) {
 #pragma unroll
                 for (int kk = 0; kk < kBwdSub / 16; ++kk) {
-                    const uint32_t acol = 32 * (kk >> 1) + 8 * (kk & 1);
-                    const uint64_t bq = smem_desc_sw128(sb + kk * 2048, kSubBytes / 2, 1024);
-                    tc_mma_ts_p(t_dk, t_dp(x) + acol, bq, idesc_g, (!first || kk > 0) ? 1u : 0u,
-                                ld);
+                    const uint32_t acol = 64 * (kk >> 2) + 8 * (kk & 3);
+                    const uint64_t bd = smem_desc_sw128(b_tile + kk * 2048, kSubBytes / 2, 1024);
+                    tc_mma_ts_p(acc, a_tm + acol, bd, idesc_g, (!first || kk > 0) ? 1u : 0u, ld);
                 }
-                tc_commit_p(bar_empty(st), ld);
             };
             for (;;) {
                 const bool got = next_item(si, false, ok, lane == 0);
@@ -479,28 +470,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     break;
                 if (!(ok = mbar_wait_warp(bar_kvfull, (uint32_t)(si & 1), abort_flag)))
                     break;
+                if (!(ok = wait_stage(g)))
+                    break;
                 tc_fence_after();
-                for (int s = 0; s <= it.nt && ok; ++s) {
-                    if (s < it.nt) {
-                        const long long gg = g + s;
-                        if (!(ok = mbar_wait_warp(bar_full((int)(gg % kKvStages)),
-                                                  (uint32_t)((gg / kKvStages) & 1), abort_flag)))
+                issue_t(t_st, base + kKvSmemK, stage(g), bar_sdone);
+                issue_t(t_dp, base + kKvSmemV, stage(g) + kSubBytes, bar_dpdone);
+                for (int s = 0; s < it.nt && ok; ++s) {
+                    const long long gg = g + s;
+                    const bool more = s + 1 < it.nt;
+                    // dV and dK of the previous item read out
+                    if (s == 0 && si >= 1 &&
+                        !(ok = mbar_wait_warp(bar_ofree, (uint32_t)((si - 1) & 1), abort_flag)))
+                        break;
+                    if (!(ok = mbar_wait_warp(bar_pready, (uint32_t)(gg & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_g(t_dv, t_st, stage(gg) + kSubBytes, s == 0);
+                    if (more) {
+                        if (!(ok = wait_stage(gg + 1)))
                             break;
                         tc_fence_after();
-                        issue_sdp(gg);
+                        issue_t(t_st, base + kKvSmemK, stage(gg + 1), bar_sdone);
                     }
-                    if (s >= 1) {
-                        const long long gp = g + s - 1;
-                        if (s == 1 && si >= 1 &&
-                            !(ok = mbar_wait_warp(bar_ofree, (uint32_t)((si - 1) & 1),
-                                                  abort_flag)))
-                            break;
-                        if (!(ok = mbar_wait_warp(bar_pfull((int)(gp & 1)),
-                                                  (uint32_t)((gp >> 1) & 1), abort_flag)))
-                            break;
-                        tc_fence_after();
-                        issue_grad(gp, s == 1);
-                    }
+                    if (!(ok = mbar_wait_warp(bar_dsready, (uint32_t)(gg & 1), abort_flag)))
+                        break;
+                    tc_fence_after();
+                    issue_g(t_dk, t_dp, stage(gg), s == 0);
+                    tc_commit_p(bar_empty((int)(gg % kKvStages)), ld);
+                    if (more)
+                        issue_t(t_dp, base + kKvSmemV, stage(gg + 1) + kSubBytes, bar_dpdone);
                 }
                 if (!ok)
                     break;
@@ -516,13 +514,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     } else {
         // ------------------------------------------ P^T, dS^T and epilogue
         // warp w: key rows 32 (w & 3) .. +31 (TMEM lane quarter), query
-        // columns 32 hc .. 32 hc + 31 of each 64-row step, hc = w >> 2.  The
-        // packed P^T / dS^T of half hc go to columns 32 hc .. 32 hc + 15 of
-        // the S^T / dP^T buffer: inside the columns this warp itself read,
-        // so the other half's loads are never overwritten.
+        // columns 64 hc .. 64 hc + 63 of each step, hc = w >> 2.  The packed
+        // P^T / dS^T of half hc go to columns 64 hc .. 64 hc + 31 of the S^T /
+        // dP^T buffer: inside the columns this warp itself read, so the other
+        // half's loads are never overwritten.
         const int wq = warp & 3, hc = warp >> 2;
         const int row = wq * 32 + lane; // key row of the tile = TMEM lane
         const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+        const uint32_t t_sth = t_st + lane_off + 64 * hc, t_dph = t_dp + lane_off + 64 * hc;
         const float sl2 = p.scale_log2;
         bool ok = true;
         long long g = 0;
@@ -535,66 +534,88 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const Span ksp = key_span(p.L, p.b, it.krow0 + min(row, it.nkeys - 1));
             for (int s = 0; s < it.nt; ++s) {
                 const long long gg = g + s;
-                const int x = (int)(gg & 1), st = (int)(gg % kKvStages);
+                const int st = (int)(gg % kKvStages);
                 int qhead, qs, rg;
                 kv_step(it, s, qhead, qs, rg);
+                // S^T ready; the stage's lse2 / D (written by the producer
+                // before its arrival on the stage barrier, which the MMA
+                // thread waited for before issuing S^T) landed
                 ok = __all_sync(0xffffffffu,
-                                mbar_wait(bar_sfull(x), (uint32_t)((gg >> 1) & 1), abort_flag));
-                if (!ok)
-                    break;
-                // the stage's lse2 / D (written by the producer before its
-                // arrival on the stage barrier, which the MMA thread waited
-                // for before issuing this step's products)
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_full(st),
-                                                       (uint32_t)((gg / kKvStages) & 1), abort_flag));
+                                mbar_wait(bar_sdone, (uint32_t)(gg & 1), abort_flag) &&
+                                    mbar_wait(bar_full(st), (uint32_t)((gg / kKvStages) & 1),
+                                              abort_flag));
                 if (!ok)
                     break;
                 tc_fence_after();
-                uint32_t sr[32], dr[32];
-                tmem_ld32x2_wait(t_st(x) + lane_off + 32 * hc, t_dp(x) + lane_off + 32 * hc, sr, dr);
                 const float *sl = reinterpret_cast<const float *>(
-                                      sbase + kKvSmemRows + st * kKvRowsBytes) + 32 * hc;
+                                      sbase + kKvSmemRows + st * kKvRowsBytes) + 64 * hc;
                 const int hi = rg == 0 ? it.hi0 : it.hi1;
                 const int flo = rg == 0 ? it.flo0 : it.flo1;
                 const int fhi = rg == 0 ? it.fhi0 : it.fhi1;
                 const bool full = qs >= flo && qs + kBwdSub <= fhi && qs + kBwdSub <= hi;
-                uint32_t mw = 0xffffffffu;
+                uint32_t mw[2] = {0xffffffffu, 0xffffffffu};
                 if (!full) {
-                    const int q0 = qs + 32 * hc;
+                    const int q0 = qs + 64 * hc;
                     const int e = min(hi, qs + kBwdSub);
                     const int lo0 = max(ksp.a0, q0) - q0, hi0 = min(ksp.a1, e) - q0;
                     const int lo1 = max(ksp.a2, q0) - q0, hi1 = min(ksp.a3, e) - q0;
-                    mw = range_bits(lo0, hi0) | range_bits(lo1, hi1);
+#pragma unroll
+                    for (int w = 0; w < 2; ++w)
+                        mw[w] = range_bits(lo0 - 32 * w, hi0 - 32 * w) |
+                                range_bits(lo1 - 32 * w, hi1 - 32 * w);
                 }
-                uint32_t pk[16], dk[16];
+                // P^T = 2^(scale log2(e) s - lse2) over the visible pairs
+                float pv[64];
+                {
+                    uint32_t sr[64], pk[32];
+                    tmem_ld32x2_wait(t_sth, t_sth + 32, sr, sr + 32);
 #pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    const float4 l4 = *reinterpret_cast<const float4 *>(sl + c);
-                    const float4 d4 = *reinterpret_cast<const float4 *>(sl + kBwdSub + c);
-                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pv[4], dv[4];
+                    for (int c = 0; c < 64; c += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4 *>(sl + c);
+                        const float la[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int cc = c + u;
-                        float xx = fmaf(__uint_as_float(sr[cc]), sl2, -la[u]);
-                        if (!((mw >> cc) & 1u))
-                            xx = -INFINITY;
-                        pv[u] = ex2(xx);
-                        dv[u] = pv[u] * (__uint_as_float(dr[cc]) - da[u]);
+                        for (int u = 0; u < 4; ++u) {
+                            const int cc = c + u;
+                            float xx = fmaf(__uint_as_float(sr[cc]), sl2, -la[u]);
+                            if (!((mw[cc >> 5] >> (cc & 31)) & 1u))
+                                xx = -INFINITY;
+                            pv[cc] = ex2(xx);
+                        }
+                        pk[c / 2] = pack_bf16x2(pv[c], pv[c + 1]);
+                        pk[c / 2 + 1] = pack_bf16x2(pv[c + 2], pv[c + 3]);
                     }
-                    pk[c / 2] = pack_bf16x2(pv[0], pv[1]);
-                    pk[c / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-                    dk[c / 2] = pack_bf16x2(dv[0], dv[1]);
-                    dk[c / 2 + 1] = pack_bf16x2(dv[2], dv[3]);
+                    tmem_st16(t_sth, pk);
+                    tmem_st16(t_sth + 16, pk + 16);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_pready);
                 }
-                tmem_st16(t_st(x) + lane_off + 32 * hc, pk);
-                tmem_st16(t_dp(x) + lane_off + 32 * hc, dk);
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(bar_pfull(x));
+                // dS^T = P^T (dP^T - D)
+                ok = __all_sync(0xffffffffu, mbar_wait(bar_dpdone, (uint32_t)(gg & 1), abort_flag));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                {
+                    uint32_t dr[64], dk[32];
+                    tmem_ld32x2_wait(t_dph, t_dph + 32, dr, dr + 32);
+#pragma unroll
+                    for (int c = 0; c < 64; c += 4) {
+                        const float4 d4 = *reinterpret_cast<const float4 *>(sl + kBwdSub + c);
+                        dk[c / 2] = pack_bf16x2(pv[c] * (__uint_as_float(dr[c]) - d4.x),
+                                                pv[c + 1] * (__uint_as_float(dr[c + 1]) - d4.y));
+                        dk[c / 2 + 1] = pack_bf16x2(pv[c + 2] * (__uint_as_float(dr[c + 2]) - d4.z),
+                                                    pv[c + 3] * (__uint_as_float(dr[c + 3]) - d4.w));
+                    }
+                    tmem_st16(t_dph, dk);
+                    tmem_st16(t_dph + 16, dk + 16);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_dsready);
+                }
             }
             if (!ok)
                 break;

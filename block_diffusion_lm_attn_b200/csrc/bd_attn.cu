@@ -530,12 +530,12 @@ bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
     p.scale = scale;
     p.scale_log2 = scale * bd::kLog2e;
 
-    CUtensorMap mq, mq64, mdo, mdo64, mk, mv;
+    CUtensorMap mq, mq_step, mdo, mdo_step, mk, mv;
     const uint64_t N = 2ull * L;
     if (!make_map_rows(&mq, q, N, (uint64_t)B * Hq, 128) ||
-        !make_map_rows(&mq64, q, N, (uint64_t)B * Hq, bd::kBwdSub) ||
+        !make_map_rows(&mq_step, q, N, (uint64_t)B * Hq, bd::kBwdSub) ||
         !make_map_rows(&mdo, dout, N, (uint64_t)B * Hq, 128) ||
-        !make_map_rows(&mdo64, dout, N, (uint64_t)B * Hq, bd::kBwdSub) ||
+        !make_map_rows(&mdo_step, dout, N, (uint64_t)B * Hq, bd::kBwdSub) ||
         !make_map_rows(&mk, k, N, (uint64_t)B * Hkv, 128) ||
         !make_map_rows(&mv, v, N, (uint64_t)B * Hkv, 128))
         return BD_ERR_CUDA;
@@ -552,8 +552,8 @@ bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
         const int G = items < G0 ? (int)items : G0;
         if (set_smem<bd::bd_bwd_dkdv_kernel>(bd::kKvSmemBytes) != BD_OK)
             return BD_ERR_CUDA;
-        bd::bd_bwd_dkdv_kernel<<<G, bd::kBwdThreads, bd::kKvSmemBytes, stream>>>(mk, mv, mq64,
-                                                                               mdo64, p);
+        bd::bd_bwd_dkdv_kernel<<<G, bd::kBwdThreads, bd::kKvSmemBytes, stream>>>(mk, mv, mq_step,
+                                                                               mdo_step, p);
         if (cudaGetLastError() != cudaSuccess)
             return BD_ERR_CUDA;
     }
