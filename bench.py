@@ -63,10 +63,10 @@ KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
     "bd_tc_pair_kernel": (
-        301162752, "e565affee58bcf47",
+        301246720, "353afd53303f9227",
         "ncu, training-shape forward, 4th launch of `bench.py --only fwd`"),
     "bd_tc_persist_kernel<1>": (
-        544057584, "e565affee58bcf47",
+        543613680, "353afd53303f9227",
         "ncu, denoise decode, median of 5 launches of `bench.py --only decode`"),
 }
 
