@@ -312,7 +312,7 @@ def run_ours(args):
         n_launch = args.steps  # one fwd kernel per step
         rows["fwd_train"] = {"tflops": round(fwd_kernel_tflops, 2),
                              "ms": round(ms, 4),
-                             "frac_of_measured_bf16":
+                             "frac_of_peak_bf16":
                                  round(fwd_kernel_tflops / tf_burst, 4)}
         if only == "all":
             e2e = run_e2e(bd, s, q, k, v, qd, kd, vd, out, lse, flush, world,
@@ -335,7 +335,7 @@ def run_ours(args):
                             n, 3, flush, world, sampler) / n
             tf = fwd_flops(sl) / (t * 1e-3) / 1e12
             rows[sl.name] = {"tflops": round(tf, 2), "ms": round(t, 4),
-                             "frac_of_measured_bf16": round(tf / tf_burst, 4)}
+                             "frac_of_peak_bf16": round(tf / tf_burst, 4)}
             del qd, kd, vd, o, ls
 
     # ---- block decode workloads (stream-K attention kernel + combine per call)
@@ -357,7 +357,7 @@ def run_ours(args):
             gbs = nbytes / (t * 1e-3) / 1e9
             rows[sd.name] = {"gbs": round(gbs, 1), "ms": round(t, 4),
                              "bytes": nbytes,
-                             "frac_of_measured_hbm": round(gbs / hbm, 4),
+                             "frac_of_peak_hbm": round(gbs / hbm, 4),
                              "frac_of_8tbs": round(gbs / 8000.0, 4)}
             if sd is bd_inputs.DEC_DENOISE:
                 dec_roof = {"bound": "hbm", "achieved": round(gbs, 1),
@@ -442,7 +442,7 @@ def extra_rows(bd, dev, flush, world, sampler, n, hbm, tf_burst):
                     n, 3, flush, world, sampler) / n
     tf = 2.5 * fwd_flops(s) / (t * 1e-3) / 1e12
     rows["bwd_train"] = {"tflops": round(tf, 2), "ms": round(t, 4),
-                         "frac_of_measured_bf16": round(tf / tf_burst, 4),
+                         "frac_of_peak_bf16": round(tf / tf_burst, 4),
                          "kernels": "row pass + dK/dV pass + dQ pass"}
     del qd, kd, vd, dod, out, lse, dq, dk, dv, ws
 
@@ -462,7 +462,7 @@ def extra_rows(bd, dev, flush, world, sampler, n, hbm, tf_burst):
               sd.B * sd.Hq * sd.b * (sd.d * 2 * 2 + 4))
     gbs = nbytes / (t * 1e-3) / 1e9
     rows["decode_cross"] = {"gbs": round(gbs, 1), "ms": round(t, 4), "bytes": nbytes,
-                            "frac_of_measured_hbm": round(gbs / hbm, 4)}
+                            "frac_of_peak_hbm": round(gbs / hbm, 4)}
 
     # sparse prefix retention of the same cache: 3/4 image tokens then text,
     # keep 0.8 of the image and all the text (alpha 0.5)
@@ -486,7 +486,7 @@ def extra_rows(bd, dev, flush, world, sampler, n, hbm, tf_burst):
     gbs = nbytes / (t * 1e-3) / 1e9
     rows["sprint_prune"] = {"gbs": round(gbs, 1), "ms": round(t, 4), "bytes": nbytes,
                             "kept_rows": kept,
-                            "frac_of_measured_hbm": round(gbs / hbm, 4)}
+                            "frac_of_peak_hbm": round(gbs / hbm, 4)}
     del qd, kcd, vcd, o, ls, wsd, ko, vo, wss
 
     # speculative step bookkeeping of the verification shape (B = 64, b = 28):
