@@ -160,6 +160,7 @@ __device__ __forceinline__ Span key_span(int L, int b, int c)
 }
 
 constexpr int kBwdSub = 128; // query rows per step of the dK/dV kernel
+static_assert(kBwdSub == 128, "the dK/dV compute warps take 64 query columns each, two per step");
 
 // Work item of the dK/dV kernel: (batch, kv-head) = w / R, rank r = w % R:
 // clean key tiles first (they are seen by the most query rows), idx
