@@ -41,3 +41,24 @@ def test_decode_bytes_count_each_visible_cache_row_once():
 def test_decode_bytes_denoise_workload():
     s = bd_inputs.DEC_DENOISE
     assert bench.decode_bytes(s, [8192] * s.B) == 547_422_208
+
+
+def test_traffic_is_quoted_only_for_the_kernel_sources_it_was_captured_on(monkeypatch):
+    # a stored ncu traffic figure belongs to one digest of the kernel
+    # sources; any other digest (the kernels changed since) quotes nothing
+    nbytes, digest, _ = bench.TRAFFIC["bd_tc_pair_kernel"]
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: digest)
+    assert bench.traffic_of("bd_tc_pair_kernel") == nbytes
+    monkeypatch.setattr(bench, "kernel_source_digest", lambda: "0" * 16)
+    assert bench.traffic_of("bd_tc_pair_kernel") is None
+    assert bench.traffic_of("no_such_kernel") is None
+
+
+def test_kernel_source_digest_covers_every_listed_source():
+    import os
+    csrc = os.path.join(bench.ROOT, "block_diffusion_lm_attn_b200", "csrc")
+    assert bench.KERNEL_SOURCES
+    for name in bench.KERNEL_SOURCES:
+        assert os.path.exists(os.path.join(csrc, name)), name
+    d = bench.kernel_source_digest()
+    assert len(d) == 16 and int(d, 16) >= 0
