@@ -4,8 +4,9 @@
 // One CTA = 4 warps = a 64-row query tile; each warp owns 16 rows.  K/V tiles
 // of 64 keys stream through a double-buffered, XOR-swizzled shared-memory
 // ring fed by 16-byte cp.async; S = QK^T and O += PV run on mma.sync; the
-// online softmax lives in registers.  Used for the split-KV block-decode
-// kernel and for head dims the tcgen05 forward kernel does not cover.
+// online softmax lives in registers.  Used for the split-KV block decode at
+// head dim 32 (the training/prefill form runs on the tcgen05 kernels at every
+// head dim, and so does the decode at 64 and 128).
 //
 // Every query row's visible key set is two intervals [a0,a1) U [a2,a3):
 //   training/prefill, noisy row of block k : [k b, k b + b) U [L, L + k b)
@@ -35,7 +36,6 @@ struct MmaParams {
     int mode;    // decode: 0 bidirectional, 1 causal inside the block
     int chunk;   // decode: keys per split
     int nsplit;  // decode: splits per (batch, kv-head)
-    int qtiles;  // fwd: 64-row query tiles per half
     float scale_log2; // softmax scale * log2(e)
 };
 
@@ -116,54 +116,35 @@ __device__ __forceinline__ Span decode_span(const MmaParams &p, const Plan &pl,
     return s;
 }
 
-template <int KIND> // 0 = training/prefill, 1 = decode split
+// the CTA's (batch, kv-head, split, row tile); false if it has no keys
 __device__ __forceinline__ bool make_plan(const MmaParams &p, Plan &pl)
 {
-    if (KIND == 0) {
-        const int bh = blockIdx.y;
-        // heaviest tiles (end of each half) first
-        int t = blockIdx.x;
-        int half = t < p.qtiles ? 1 : 0;
-        int idx = p.qtiles - 1 - (t < p.qtiles ? t : t - p.qtiles);
-        int r0 = (half ? p.L : 0) + idx * kMmaBM;
-        pl.nrows = min(kMmaBM, p.L - idx * kMmaBM);
-        Span first = fwd_span(p.L, p.b, r0);
-        Span last = fwd_span(p.L, p.b, r0 + pl.nrows - 1);
-        pl.lo[0] = first.a0; pl.hi[0] = last.a1;
-        pl.lo[1] = first.a2; pl.hi[1] = last.a3;
-        pl.flo[0] = last.a0; pl.fhi[0] = first.a1;
-        pl.flo[1] = last.a2; pl.fhi[1] = first.a3;
-        pl.row0 = r0;
-        pl.gbase = bh;
-        return true;
-    } else {
-        const int unit = blockIdx.z; // batch * Hkv + kv-head
-        const int bi = unit / p.Hkv, g = unit % p.Hkv;
-        const int group = p.Hq / p.Hkv;
-        const int len = p.cache_len[bi];
-        const int s = blockIdx.x;
-        const int own = p.mode == 2 ? 0 : p.b; // keys past the prefix
-        if (len < 0 || (long long)len + own > p.nkeys)
-            return false; // reported by the combine kernel
-        const int total = len + own;
-        if (s * p.chunk >= total)
-            return false;
-        pl.len = len;
-        pl.split = s;
-        pl.row0 = blockIdx.y * kMmaBM;
-        pl.nrows = min(kMmaBM, group * p.b - pl.row0);
-        pl.gbase = (bi * p.Hq + g * group) * p.b; // global row of local row 0
-        const int s0 = s * p.chunk, s1 = min(total, s0 + p.chunk);
-        pl.lo[0] = s0; pl.hi[0] = s1;
-        pl.lo[1] = 0; pl.hi[1] = 0;
-        pl.flo[0] = s0;
-        pl.fhi[0] = min(s1, len + (p.mode == 0 ? p.b : 0));
-        pl.flo[1] = 0; pl.fhi[1] = 0;
-        return true;
-    }
+    const int unit = blockIdx.z; // batch * Hkv + kv-head
+    const int bi = unit / p.Hkv, g = unit % p.Hkv;
+    const int group = p.Hq / p.Hkv;
+    const int len = p.cache_len[bi];
+    const int s = blockIdx.x;
+    const int own = p.mode == 2 ? 0 : p.b; // keys past the prefix
+    if (len < 0 || (long long)len + own > p.nkeys)
+        return false; // reported by the combine kernel
+    const int total = len + own;
+    if (s * p.chunk >= total)
+        return false;
+    pl.len = len;
+    pl.split = s;
+    pl.row0 = blockIdx.y * kMmaBM;
+    pl.nrows = min(kMmaBM, group * p.b - pl.row0);
+    pl.gbase = (bi * p.Hq + g * group) * p.b; // global row of local row 0
+    const int s0 = s * p.chunk, s1 = min(total, s0 + p.chunk);
+    pl.lo[0] = s0; pl.hi[0] = s1;
+    pl.lo[1] = 0; pl.hi[1] = 0;
+    pl.flo[0] = s0;
+    pl.fhi[0] = min(s1, len + (p.mode == 0 ? p.b : 0));
+    pl.flo[1] = 0; pl.fhi[1] = 0;
+    return true;
 }
 
-template <int D, int KIND>
+template <int D>
 __global__ void __launch_bounds__(kMmaThreads)
     bd_mma_attn_kernel(const MmaParams p)
 {
@@ -173,24 +154,13 @@ __global__ void __launch_bounds__(kMmaThreads)
     bf16 *sV = sK + 2 * kMmaBM * D;
 
     Plan pl;
-    if (!make_plan<KIND>(p, pl))
+    if (!make_plan(p, pl))
         return;
 
-    const bf16 *qsrc, *kbase, *vbase;
-    if (KIND == 0) {
-        const size_t N = 2 * (size_t)p.L;
-        const int bh = blockIdx.y;
-        const int bi = bh / p.Hq, h = bh % p.Hq;
-        const int g = h / (p.Hq / p.Hkv);
-        qsrc = p.q + ((size_t)bh * N + pl.row0) * D;
-        kbase = p.k + (size_t)(bi * p.Hkv + g) * N * D;
-        vbase = p.v + (size_t)(bi * p.Hkv + g) * N * D;
-    } else {
-        const int unit = blockIdx.z;
-        qsrc = p.q + ((size_t)pl.gbase + pl.row0) * D;
-        kbase = p.k + (size_t)unit * p.nkeys * D;
-        vbase = p.v + (size_t)unit * p.nkeys * D;
-    }
+    const int unit = blockIdx.z;
+    const bf16 *qsrc = p.q + ((size_t)pl.gbase + pl.row0) * D;
+    const bf16 *kbase = p.k + (size_t)unit * p.nkeys * D;
+    const bf16 *vbase = p.v + (size_t)unit * p.nkeys * D;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;
@@ -200,8 +170,7 @@ __global__ void __launch_bounds__(kMmaThreads)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
         int rl = min(warp * 16 + gq + 8 * i, pl.nrows - 1);
-        sp[i] = (KIND == 0) ? fwd_span(p.L, p.b, pl.row0 + rl)
-                            : decode_span(p, pl, rl);
+        sp[i] = decode_span(p, pl, rl);
     }
 
     // key tiles: range 0 then range 1
@@ -358,30 +327,17 @@ __global__ void __launch_bounds__(kMmaThreads)
             continue;
         const float inv = l[i] > 0.f ? 1.f / l[i] : 0.f;
         const float lse = l[i] > 0.f ? (m[i] + __log2f(l[i])) * kLn2 : -INFINITY;
-        if (KIND == 0) {
-            const size_t row = (size_t)pl.gbase * 2 * p.L + pl.row0 + rl;
-            bf16 *orow = p.out + row * D;
+        const size_t rows_all = (size_t)p.B * p.Hq * p.b;
+        const size_t row = (size_t)pl.gbase + pl.row0 + rl;
+        float *orow = p.part_o + ((size_t)pl.split * rows_all + row) * D;
 #pragma unroll
-            for (int nt8 = 0; nt8 < D / 8; ++nt8) {
-                uint32_t v2 = pack_bf16x2(o[nt8][2 * i] * inv,
-                                          o[nt8][2 * i + 1] * inv);
-                *reinterpret_cast<uint32_t *>(orow + nt8 * 8 + 2 * tq) = v2;
-            }
-            if (tq == 0)
-                p.lse[row] = lse;
-        } else {
-            const size_t rows_all = (size_t)p.B * p.Hq * p.b;
-            const size_t row = (size_t)pl.gbase + pl.row0 + rl;
-            float *orow = p.part_o + ((size_t)pl.split * rows_all + row) * D;
-#pragma unroll
-            for (int nt8 = 0; nt8 < D / 8; ++nt8) {
-                float2 v2 = make_float2(o[nt8][2 * i] * inv,
-                                        o[nt8][2 * i + 1] * inv);
-                *reinterpret_cast<float2 *>(orow + nt8 * 8 + 2 * tq) = v2;
-            }
-            if (tq == 0)
-                p.part_lse[(size_t)pl.split * rows_all + row] = lse;
+        for (int nt8 = 0; nt8 < D / 8; ++nt8) {
+            float2 v2 = make_float2(o[nt8][2 * i] * inv,
+                                    o[nt8][2 * i + 1] * inv);
+            *reinterpret_cast<float2 *>(orow + nt8 * 8 + 2 * tq) = v2;
         }
+        if (tq == 0)
+            p.part_lse[(size_t)pl.split * rows_all + row] = lse;
     }
 }
 

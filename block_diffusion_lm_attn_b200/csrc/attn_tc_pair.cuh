@@ -90,8 +90,9 @@ __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
     sg.nt = sg.n0 + n1;
 }
 
-// DH: head dim of the tensors, 128, or 64 read zero-extended to 128 columns
-// (the QKs skip the zero half; the upper 64 columns of O are never written).
+// DH: head dim of the tensors, 128, or 64 / 32 read zero-extended to 128
+// columns (the QKs skip the zero K-steps; the columns of O past DH are never
+// written).
 template <int DH>
 __global__ void __launch_bounds__(kPairThreads, 1)
     bd_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 const uint32_t ts = tmem + (uint32_t)x * 128;
 #pragma unroll
                 for (int kk = 0; kk < kTcD / 16; ++kk) {
-                    if (kk * 16 >= DH) // zero columns of a head dim of 64
+                    if (kk * 16 >= DH) // zero columns of a head dim below 128
                         break;
                     const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                     tc_mma_ss_p(ts, smem_desc_sw128(qb + off, 16, 1024),
@@ -446,6 +447,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const int q4 = 2 * h + q;
+                    if (q4 * 32 >= DH)
+                        break;
                     uint32_t o[32];
                     tmem_ld32_wait(t_o + lane_off + q4 * 32, o);
 #pragma unroll
@@ -472,7 +475,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                  : "r"(epi + (uint32_t)r * 128 + ((cc ^ (uint32_t)(r & 7)) << 4))
                                  : "memory");
                     const int trow = wq * 32 + r;
-                    if (trow < sg.nrows)
+                    if (trow < sg.nrows && h * 64 + (int)cc * 8 < DH)
                         reinterpret_cast<uint4 *>(p.out + (head_row0 + trow) * DH)[h * 8 + cc] =
                             make_uint4(x0, x1, x2, x3);
                 }

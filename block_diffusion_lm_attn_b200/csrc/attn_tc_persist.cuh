@@ -258,8 +258,9 @@ struct DecSource {
 // ----------------------------------------------------------------------------
 
 // KIND 0: training/prefill form, 1: block decode.  DH: head dim of the
-// tensors, 128, or 64 read zero-extended to 128 columns (the QKs skip the zero
-// half; the upper 64 columns of O are computed but never written out).
+// tensors, 128, or 64 / 32 read zero-extended to 128 columns (the QKs skip
+// the zero K-steps; the columns of O past DH are computed but never written
+// out).  Head dim 32 runs here for the training/prefill form only.
 template <int KIND, int DH>
 __global__ void __launch_bounds__(kTcThreads, 1)
     bd_tc_persist_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     const uint32_t ts = t_s0 + (uint32_t)b * 128;
 #pragma unroll
                     for (int kk = 0; kk < kTcD / 16; ++kk) {
-                        if (kk * 16 >= DH) // zero columns of a head dim of 64
+                        if (kk * 16 >= DH) // zero columns of a head dim below 128
                             break;
                         const uint32_t off = (kk >> 2) * kHalfTileBytes + (kk & 3) * 32;
                         tc_mma_ss(ts, smem_desc_sw128(qb + off, 16, 1024),

@@ -67,7 +67,8 @@ bool pair_kernel_usable()
 
 bool pair_kernel_usable(int d)
 {
-    return d == 64 ? pair_kernel_usable<64>() : pair_kernel_usable<128>();
+    return d == 64 ? pair_kernel_usable<64>()
+                   : d == 32 ? pair_kernel_usable<32>() : pair_kernel_usable<128>();
 }
 
 // Grid cap set by bd_attn_debug_set_grid (0: none).
@@ -263,29 +264,20 @@ bd_status launch_persist(const CUtensorMap &mq, const CUtensorMap &mk,
                          const CUtensorMap &mv, const bd::PParams &p, int grid,
                          cudaStream_t st)
 {
+    if constexpr (KIND == 0) // head dim 32 decodes on the split-KV kernel
+        if (p.d == 32)
+            return launch_persist_dh<KIND, 32>(mq, mk, mv, p, grid, st);
     return p.d == 64 ? launch_persist_dh<KIND, 64>(mq, mk, mv, p, grid, st)
                      : launch_persist_dh<KIND, 128>(mq, mk, mv, p, grid, st);
-}
-
-template <int D>
-bd_status launch_fwd_mma(const bd::MmaParams &p, cudaStream_t st)
-{
-    auto kern = bd::bd_mma_attn_kernel<D, 0>;
-    constexpr int smem = bd::mma_smem_bytes<D>();
-    if (set_smem<bd::bd_mma_attn_kernel<D, 0>>(smem) != BD_OK)
-        return BD_ERR_CUDA;
-    dim3 grid(2 * p.qtiles, p.B * p.Hq);
-    kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
 }
 
 template <int D>
 bd_status launch_decode_mma(const bd::MmaParams &p, const DecodePlan &pl,
                             cudaStream_t st)
 {
-    auto kern = bd::bd_mma_attn_kernel<D, 1>;
+    auto kern = bd::bd_mma_attn_kernel<D>;
     constexpr int smem = bd::mma_smem_bytes<D>();
-    if (set_smem<bd::bd_mma_attn_kernel<D, 1>>(smem) != BD_OK)
+    if (set_smem<bd::bd_mma_attn_kernel<D>>(smem) != BD_OK)
         return BD_ERR_CUDA;
     dim3 grid(pl.nsplit, pl.row_tiles, p.B * p.Hkv);
     kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
@@ -394,10 +386,7 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
     p.chunk = pl.chunk;
     p.nsplit = pl.nsplit;
     p.scale_log2 = scale_log2;
-    switch (d) {
-    case 32: return launch_decode_mma<32>(p, pl, stream);
-    default: return launch_decode_mma<64>(p, pl, stream);
-    }
+    return launch_decode_mma<32>(p, pl, stream); // the only head dim decoded here
 }
 
 } // namespace
@@ -437,8 +426,9 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
     if ((long long)B * Hq > 65535LL || 2LL * L * (long long)B * Hq * d > (1LL << 40))
         return BD_ERR_UNSUPPORTED;
 
-    if (d == 128 || d == 64) {
-        // tcgen05 kernels; d = 64 runs on tiles zero-extended to 128 columns
+    {
+        // tcgen05 kernels; d = 64 and 32 run on tiles zero-extended to 128
+        // columns
         bd::PParams p = {};
         p.out = static_cast<bf16 *>(out);
         p.lse = lse;
@@ -461,24 +451,10 @@ bd_status bd_attn_fwd(const void *q, const void *k, const void *v, void *out,
         if (items < G)
             G = (int)items;
         if (pair)
-            return d == 64 ? launch_pair<64>(mq, mk, mv, p, G, stream)
-                           : launch_pair<128>(mq, mk, mv, p, G, stream);
+            return d == 64   ? launch_pair<64>(mq, mk, mv, p, G, stream)
+                   : d == 32 ? launch_pair<32>(mq, mk, mv, p, G, stream)
+                             : launch_pair<128>(mq, mk, mv, p, G, stream);
         return launch_persist<0>(mq, mk, mv, p, G, stream);
-    }
-
-    bd::MmaParams p = {};
-    p.q = static_cast<const bf16 *>(q);
-    p.k = static_cast<const bf16 *>(k);
-    p.v = static_cast<const bf16 *>(v);
-    p.out = static_cast<bf16 *>(out);
-    p.lse = lse;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
-    p.nkeys = 2 * L;
-    p.qtiles = (int)cdiv(L, bd::kMmaBM);
-    p.scale_log2 = scale * bd::kLog2e;
-    switch (d) {
-    case 32: return launch_fwd_mma<32>(p, stream);
-    default: return launch_fwd_mma<64>(p, stream);
     }
 }
 
@@ -727,8 +703,6 @@ int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d)
 {
     if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !supported_d(d))
         return -1;
-    if (d == 32)
-        return 0;
     return ((Hq / Hkv) % 2 == 0 && pair_kernel_usable(d)) ? 2 : 1;
 }
 

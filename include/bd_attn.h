@@ -79,10 +79,10 @@ typedef enum {
  * BD_ERR_UNSUPPORTED for d not in {32, 64, 128}; BD_ERR_CUDA if the launch
  * fails.
  *
- * Kernels: d = 128 and d = 64 run on the tcgen05 / TMA kernels (d = 64 on
- * tiles read zero-extended to 128 columns); d = 32 on an mma.sync kernel.
+ * Kernels: every head dim runs on the tcgen05 / TMA kernels (d = 64 and 32
+ * on tiles read zero-extended to 128 columns).
  *
- * Concurrency (d = 128, 64): the launch is one persistent CTA per SM that takes
+ * Concurrency: the launch is one persistent CTA per SM that takes
  * its work items from one of 64 counter pairs in device memory, chosen
  * round-robin when the call is made (and so fixed inside a captured CUDA
  * graph) and reset by the launch's last CTA.  Launches sharing a pair must

@@ -43,10 +43,11 @@ BD_API bd_status bd_attn_debug_set_grid(int ctas);
 
 /*
  * Which kernel bd_attn_fwd runs for these sizes on the current device:
- * 2 = tcgen05 kernel with two query heads of a GQA group per CTA (d = 128
- * or 64, even group size), 1 = tcgen05 kernel with one query tile per CTA
- * (d = 128 or 64, odd group size, or the paired kernel's register split
- * unavailable), 0 = mma.sync kernel (d = 32), -1 = sizes bd_attn_fwd rejects.
+ * 2 = tcgen05 kernel with two query heads of a GQA group per CTA (even group
+ * size), 1 = tcgen05 kernel with one query tile per CTA (odd group size, or
+ * the paired kernel's register split unavailable), -1 = sizes bd_attn_fwd
+ * rejects.  (0, an mma.sync kernel, is no longer returned: every head dim
+ * runs on the tcgen05 kernels.)
  * Needs the CUDA runtime (it reads the compiled kernel's attributes).
  */
 BD_API int bd_attn_debug_fwd_kernel(int Hq, int Hkv, int d);

@@ -86,20 +86,23 @@ FWD_GRID = [
     (1, 4, 1, 512, 512, 128),   # one block per half (b = L)
     (1, 4, 2, 200, 8, 64),      # head dim 64 on the paired kernel, ragged tails
     (2, 3, 3, 136, 17, 64),     # head dim 64 on the one-tile kernel
+    (1, 4, 2, 200, 8, 32),      # head dim 32 on the paired kernel, ragged tails
+    (2, 3, 3, 136, 17, 32),     # head dim 32 on the one-tile kernel
 ]
 
 
 def test_fwd_kernel_selection():
-    """Even GQA groups of head dim 128 or 64 run the paired tcgen05 kernel
-    (the one the benchmark times), odd groups the one-tile tcgen05 kernel,
-    head dim 32 the mma.sync kernel; so the grid below covers each."""
+    """Even GQA groups run the paired tcgen05 kernel (the one the benchmark
+    times), odd groups the one-tile tcgen05 kernel, at every head dim; so the
+    grid below covers each kernel at 128, 64 and 32."""
     assert bd.bd_attn_debug_fwd_kernel(32, 8, 128) == 2
     assert bd.bd_attn_debug_fwd_kernel(4, 2, 128) == 2
     assert bd.bd_attn_debug_fwd_kernel(8, 8, 128) == 1
     assert bd.bd_attn_debug_fwd_kernel(3, 1, 128) == 1
     assert bd.bd_attn_debug_fwd_kernel(4, 2, 64) == 2
     assert bd.bd_attn_debug_fwd_kernel(2, 2, 64) == 1
-    assert bd.bd_attn_debug_fwd_kernel(2, 2, 32) == 0
+    assert bd.bd_attn_debug_fwd_kernel(4, 2, 32) == 2
+    assert bd.bd_attn_debug_fwd_kernel(2, 2, 32) == 1
     assert bd.bd_attn_debug_fwd_kernel(3, 2, 128) == -1
 
 
