@@ -59,7 +59,7 @@ HOST_COVER_CYCLES = 400000  # ~0.2 ms GPU sleep queued before each timed step
 # captured with; if the sources differ now, the figure no longer describes the
 # kernel and the bench reports traffic as null.
 KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
-                  "attn_mma.cuh", "bd_common.cuh")
+                  "bd_mask.cuh", "bd_common.cuh")
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
     "bd_tc_pair_kernel": (

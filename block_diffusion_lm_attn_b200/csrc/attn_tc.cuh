@@ -21,7 +21,7 @@
 
 #include <cuda.h>
 
-#include "attn_mma.cuh"
+#include "bd_mask.cuh"
 #include "bd_common.cuh"
 
 namespace bd {

@@ -260,7 +260,7 @@ struct DecSource {
 // KIND 0: training/prefill form, 1: block decode.  DH: head dim of the
 // tensors, 128, or 64 / 32 read zero-extended to 128 columns (the QKs skip
 // the zero K-steps; the columns of O past DH are computed but never written
-// out).  Head dim 32 runs here for the training/prefill form only.
+// out).
 template <int KIND, int DH>
 __global__ void __launch_bounds__(kTcThreads, 1)
     bd_tc_persist_kernel(const __grid_constant__ CUtensorMap tm_q,

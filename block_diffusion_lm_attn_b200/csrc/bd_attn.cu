@@ -17,7 +17,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include "attn_mma.cuh"
 #include "attn_tc.cuh"
 #include "attn_tc_persist.cuh"
 #include "attn_tc_pair.cuh"
@@ -88,15 +87,12 @@ int persistent_grid()
 }
 
 // Decode launch plan.  A pure function of the sizes, so the workspace query
-// and the launch agree without a device round trip.
-//   d = 128 or 64: stream-K over (unit, key tile) on <= kMaxGrid persistent
-//            CTAs (d = 64 on tiles zero-extended to 128 columns); scratch =
-//            2 partial (o, lse) slots of 128 rows x 128 columns per CTA.
-//   d = 32:  split-KV with `nsplit` chunks of `chunk` keys per (sequence,
-//            kv-head, 64-row tile); scratch = nsplit partials per row.
+// and the launch agree without a device round trip: stream-K over (unit, key
+// tile) on <= kMaxGrid persistent CTAs (d = 64 and 32 on tiles zero-extended
+// to 128 columns); scratch = 2 partial (o, lse) slots of 128 rows x 128
+// columns per CTA and a cut descriptor per CTA, whatever the sizes.
 struct DecodePlan {
-    bool tc;
-    int row_tiles, nsplit, chunk;
+    int row_tiles;
     size_t rows_all, o_bytes, lse_bytes, desc_bytes, total_bytes;
 };
 
@@ -108,29 +104,10 @@ bool decode_plan(int B, int Hq, int Hkv, int b, int d, int S_cap,
         return false;
     const long long rows = (long long)(Hq / Hkv) * b;
     pl.rows_all = (size_t)B * Hq * b;
-    pl.tc = (d == 128 || d == 64);
-    if (pl.tc) {
-        pl.row_tiles = (int)cdiv(rows, bd::kTcM);
-        pl.nsplit = 0;
-        pl.chunk = 0;
-        pl.o_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * bd::kTcD * sizeof(float));
-        pl.lse_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * sizeof(float));
-        pl.desc_bytes = round256((size_t)kMaxGrid * sizeof(int4));
-    } else {
-        pl.row_tiles = (int)cdiv(rows, bd::kMmaBM);
-        const long long units = (long long)B * Hkv * pl.row_tiles;
-        const long long target = 4LL * kMaxGrid;
-        long long ns = cdiv(target, units);
-        const long long max_ns = cdiv(S_cap, 256);
-        if (ns > max_ns) ns = max_ns;
-        if (ns < 1) ns = 1;
-        const long long chunk = cdiv(cdiv(S_cap, ns), 64) * 64;
-        pl.chunk = (int)chunk;
-        pl.nsplit = (int)cdiv(S_cap, chunk);
-        pl.o_bytes = round256((size_t)pl.nsplit * pl.rows_all * d * sizeof(float));
-        pl.lse_bytes = round256((size_t)pl.nsplit * pl.rows_all * sizeof(float));
-        pl.desc_bytes = 0;
-    }
+    pl.row_tiles = (int)cdiv(rows, bd::kTcM);
+    pl.o_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * bd::kTcD * sizeof(float));
+    pl.lse_bytes = round256((size_t)kMaxGrid * 2 * bd::kTcM * sizeof(float));
+    pl.desc_bytes = round256((size_t)kMaxGrid * sizeof(int4));
     pl.total_bytes = pl.o_bytes + pl.lse_bytes + pl.desc_bytes;
     return true;
 }
@@ -264,28 +241,9 @@ bd_status launch_persist(const CUtensorMap &mq, const CUtensorMap &mk,
                          const CUtensorMap &mv, const bd::PParams &p, int grid,
                          cudaStream_t st)
 {
-    if constexpr (KIND == 0) // head dim 32 decodes on the split-KV kernel
-        if (p.d == 32)
-            return launch_persist_dh<KIND, 32>(mq, mk, mv, p, grid, st);
-    return p.d == 64 ? launch_persist_dh<KIND, 64>(mq, mk, mv, p, grid, st)
-                     : launch_persist_dh<KIND, 128>(mq, mk, mv, p, grid, st);
-}
-
-template <int D>
-bd_status launch_decode_mma(const bd::MmaParams &p, const DecodePlan &pl,
-                            cudaStream_t st)
-{
-    auto kern = bd::bd_mma_attn_kernel<D>;
-    constexpr int smem = bd::mma_smem_bytes<D>();
-    if (set_smem<bd::bd_mma_attn_kernel<D>>(smem) != BD_OK)
-        return BD_ERR_CUDA;
-    dim3 grid(pl.nsplit, pl.row_tiles, p.B * p.Hkv);
-    kern<<<grid, bd::kMmaThreads, smem, st>>>(p);
-    if (cudaGetLastError() != cudaSuccess)
-        return BD_ERR_CUDA;
-    const int rows_all = p.B * p.Hq * p.b;
-    bd::bd_decode_combine_kernel<D><<<(rows_all + 7) / 8, 256, 0, st>>>(p);
-    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+    return p.d == 64   ? launch_persist_dh<KIND, 64>(mq, mk, mv, p, grid, st)
+           : p.d == 32 ? launch_persist_dh<KIND, 32>(mq, mk, mv, p, grid, st)
+                       : launch_persist_dh<KIND, 128>(mq, mk, mv, p, grid, st);
 }
 
 // Host-side checks shared by both decode entry points.
@@ -330,7 +288,7 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
     float *part_lse =
         reinterpret_cast<float *>(static_cast<char *>(workspace) + pl.o_bytes);
     const float scale_log2 = (1.0f / std::sqrt((float)d)) * bd::kLog2e;
-    if (pl.tc) {
+    {
         bd::PParams p = {};
         p.out = static_cast<bf16 *>(out);
         p.lse = lse;
@@ -371,22 +329,6 @@ bd_status decode_launch(const void *q_blk, const void *k_cache,
             return BD_ERR_CUDA;
         return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
     }
-    bd::MmaParams p = {};
-    p.q = static_cast<const bf16 *>(q_blk);
-    p.k = static_cast<const bf16 *>(k_cache);
-    p.v = static_cast<const bf16 *>(v_cache);
-    p.out = static_cast<bf16 *>(out);
-    p.lse = lse;
-    p.part_o = part_o;
-    p.part_lse = part_lse;
-    p.cache_len = cache_len;
-    p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = 0; p.b = b;
-    p.nkeys = S_cap;
-    p.mode = mode;
-    p.chunk = pl.chunk;
-    p.nsplit = pl.nsplit;
-    p.scale_log2 = scale_log2;
-    return launch_decode_mma<32>(p, pl, stream); // the only head dim decoded here
 }
 
 } // namespace
@@ -751,6 +693,12 @@ bd_status bd_attn_get_device_status(cudaStream_t stream)
 
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[BD_ATTN_NOALLOC_SCRATCH_BYTES];
+// the decode scratch is the same for every size (decode_plan); it fits
+static_assert(2 * kMaxGrid * bd::kTcM * bd::kTcD * sizeof(float) +
+                      2 * kMaxGrid * bd::kTcM * sizeof(float) + kMaxGrid * sizeof(int4) +
+                      3 * 256 <=
+                  BD_ATTN_NOALLOC_SCRATCH_BYTES,
+              "the fixed no-alloc array must hold the decode scratch");
 
 namespace {
 

@@ -173,14 +173,13 @@ BD_API size_t bd_attn_bwd_workspace_bytes(int B, int Hq, int L);
  *   S_cap            row capacity of the caches (>= b in modes 0 and 1)
  *   workspace        device scratch of at least
  *                    bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d, S_cap)
- *                    bytes, 256-byte aligned, used for the split-KV partial
- *                    results; its contents on entry do not matter.  NULL
- *                    makes the library use an internal buffer of the current
- *                    device: a call that needs more than the current one
- *                    allocates a larger buffer (so that call must not be
- *                    inside a stream capture); buffers handed out are never
- *                    freed, so graphs captured with an earlier one stay
- *                    valid.  Every NULL-workspace call on a device shares
+ *                    bytes (19.6 MB, the same for every size: the partial
+ *                    results of at most two cut units per persistent CTA),
+ *                    256-byte aligned; its contents on entry do not matter.
+ *                    NULL makes the library use an internal buffer of the
+ *                    current device, allocated by the first such call (so
+ *                    that call must not be inside a stream capture) and
+ *                    never freed, so graphs captured with it stay valid.  Every NULL-workspace call on a device shares
  *                    the current buffer: calls whose kernels may overlap on
  *                    the GPU (two streams without ordering between them)
  *                    race on it and give wrong results -- order them, or
@@ -215,16 +214,16 @@ BD_API bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
  * inside a stream capture where allocation is not allowed, or real-time code
  * that forbids allocation after start-up.  This call computes exactly what
  * bd_attn_decode computes, with the same arguments, layouts and errors, but
- * takes no workspace: its split-KV scratch is a fixed array of
- * BD_ATTN_NOALLOC_SCRATCH_BYTES bytes compiled into the library's device
- * code.  Every GPU on which the library's kernels are loaded holds that array
+ * takes no workspace: its scratch (bd_attn_decode_workspace_bytes, 19.6 MB
+ * for every size) lives in a fixed array of BD_ATTN_NOALLOC_SCRATCH_BYTES
+ * bytes compiled into the library's device code.  Every GPU on which the library's kernels are loaded holds that array
  * until the process exits.
  *
  * - The first call on a device looks up the array's device address (with
  *   that device current) and caches it; make that first call before any
  *   stream capture.
- * - Sizes whose scratch, bd_attn_decode_workspace_bytes(B, Hq, Hkv, b, d,
- *   S_cap), exceeds BD_ATTN_NOALLOC_SCRATCH_BYTES are rejected with
+ * - The array holds the scratch of every size (checked when the library is
+ *   built); a size whose scratch exceeded it would be rejected with
  *   BD_ERR_UNSUPPORTED before anything is launched.
  * - All calls share the one array and it keeps whatever the last call left
  *   there; nothing in it needs to start at zero.  Calls whose kernels overlap

@@ -49,6 +49,15 @@ def test_workspace_bytes(lib):
     assert bd.bd_attn_decode_workspace_bytes(1, 4, 4, 32, 128, 16) > 0
     w = bd.bd_attn_decode_workspace_bytes(16, 32, 8, 32, 128, 8224)
     assert w % 256 == 0
+    # stream-K scratch: two (o, lse) slots of 128 x 128 fp32 rows and a cut
+    # descriptor per persistent CTA (148), whatever the sizes and head dim
+    per = 2 * 148 * 128 * 128 * 4 + 2 * 148 * 128 * 4 + 148 * 16
+    assert per <= w < per + 3 * 256
+    for args in [(1, 4, 4, 8, 32, 64), (256, 64, 8, 32, 32, 65536),
+                 (64, 32, 8, 28, 64, 8224), (3, 8, 2, 16, 128, 20)]:
+        assert bd.bd_attn_decode_workspace_bytes(*args) == w, args
+    # the no-alloc entry point's fixed array holds it
+    assert w <= 32 << 20
 
 
 A = 1 << 20  # a 16-byte-aligned fake address; never dereferenced

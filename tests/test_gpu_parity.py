@@ -287,10 +287,11 @@ def test_decode_bad_cache_len_is_reported():
     check(out[:1], lse[:1], ro, rl, "good sequence next to a bad one")
 
 
-def test_internal_workspace_survives_growth_under_a_captured_graph():
+def test_internal_workspace_under_a_captured_graph():
     """A graph captured with the library's internal decode workspace
-    (workspace = NULL) stays valid after a later call needs a larger
-    internal workspace: the earlier buffer is kept, not freed."""
+    (workspace = NULL) replays correctly after other NULL-workspace calls,
+    of other sizes and head dims, ran in between: the buffer is allocated
+    once per device, is the same size for every call, and is never freed."""
     B, Hq, Hkv, b, d = 4, 32, 8, 32, 128
     lens = [900, 17, 2048, 511]
     S_cap = 2100
@@ -308,17 +309,17 @@ def test_internal_workspace_survives_growth_under_a_captured_graph():
         with torch.cuda.graph(g, stream=s):
             bd.decode(qd, kd, vd, cd, 0, out=out, lse=lse, stream=s)
     torch.cuda.synchronize()
-    # a head-dim-32 call whose split-KV scratch exceeds the current buffer
-    B2, Hq2, Hkv2, b2, d2 = 256, 32, 8, 32, 32
-    assert (bd.workspace_bytes(B2, Hq2, Hkv2, b2, d2, 64) >
-            bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap))
-    q2, kc2, vc2, cl2 = bd_inputs.decode_inputs(B2, Hq2, Hkv2, b2, d2, 64,
-                                                cache_len=[20] * B2, seed=24)
-    bd.decode(q2.cuda(), kc2.cuda(), vc2.cuda(), cl2.cuda(), 1)
+    # other sizes and head dims through the same internal buffer
+    for (B2, Hq2, Hkv2, b2, d2, n) in [(256, 32, 8, 32, 32, 20), (3, 4, 1, 8, 64, 300)]:
+        assert bd.workspace_bytes(B2, Hq2, Hkv2, b2, d2, n + b2) == \
+            bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap)
+        q2, kc2, vc2, cl2 = bd_inputs.decode_inputs(B2, Hq2, Hkv2, b2, d2, n + b2,
+                                                    cache_len=[n] * B2, seed=24)
+        bd.decode(q2.cuda(), kc2.cuda(), vc2.cuda(), cl2.cuda(), 1)
     torch.cuda.synchronize()
     out.zero_()
     g.replay()
     torch.cuda.synchronize()
     assert bd.device_status() == bd.BD_OK
     ro, rl = oracle.decode(q, kc, vc, cl, 0, 1 / math.sqrt(d))
-    check(out, lse, ro, rl, "graph replay after workspace growth")
+    check(out, lse, ro, rl, "graph replay after other calls on the internal workspace")

@@ -1,11 +1,9 @@
 """Block decode through bd_attn_decode_noalloc, the entry point for callers
-that cannot allocate device memory at decode time (its split-KV scratch is a
-fixed array inside the library).  Two calls in a row, with different inputs,
-each compared with bd_attn_decode on the same inputs, and once directly with
-the fp64 oracle; both scratch layouts (the stream-K layout of the tcgen05
-kernel, d = 128 and 64, and the split-KV layout of the d = 32 kernel share
-the array); and a call inside a captured CUDA
-graph in global capture mode, where any allocation would fail the capture.
+that cannot allocate device memory at decode time (its scratch is a fixed
+array inside the library).  Calls in a row at head dims 128, 64 and 32, with
+different inputs, each compared with bd_attn_decode on the same inputs, and
+once directly with the fp64 oracle; and a call inside a captured CUDA graph
+in global capture mode, where any allocation would fail the capture.
 Collected last so that a run stopping at the first failure has already run
 every other test."""
 import math
@@ -22,7 +20,6 @@ from block_diffusion_lm_attn_b200 import build
 pytestmark = pytest.mark.gpu
 
 OUT_MAX, OUT_MEAN, LSE_MAX = 2e-2, 2e-3, 1e-3
-SCRATCH_MAX = 32 << 20
 
 
 def _call_noalloc(q, kc, vc, cl, mode, out, lse):
@@ -56,7 +53,7 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
     bd.load()
     for B, Hq, Hkv, b, d, lens, mode in CASES:
         S_cap = max(lens) + b
-        assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) <= SCRATCH_MAX
+        assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) <= 32 << 20  # the fixed array
         q, kc, vc, cl = bd_inputs.decode_inputs(B, Hq, Hkv, b, d, S_cap,
                                                 cache_len=lens, seed=B + b)
         q, kc, vc, cl = q.cuda(), kc.cuda(), vc.cuda(), cl.cuda()
@@ -67,14 +64,6 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
         torch.cuda.synchronize()
         assert bd.device_status() == bd.BD_OK
         _compare(ref_o, ref_l, out, lse)
-
-    # a size whose scratch exceeds the fixed array is refused up front
-    B, Hq, Hkv, b, d, S_cap = 256, 64, 8, 32, 32, 65536
-    assert bd.workspace_bytes(B, Hq, Hkv, b, d, S_cap) > SCRATCH_MAX
-    A = 1 << 20
-    st = bd.bd_attn_decode_noalloc(A, A, A, A, A, A, B, Hq, Hkv, b, d, 0,
-                                   None, S_cap)
-    assert st == bd.BD_ERR_UNSUPPORTED
 
 
 def test_noalloc_decode_matches_the_oracle():
