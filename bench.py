@@ -63,10 +63,10 @@ KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
     "bd_tc_pair_kernel": (
-        300966400, "0f1dbc2f5b303f37",
+        301016064, "cde748c09c00bdc2",
         "ncu, training-shape forward, 4th launch of `bench.py --only fwd`"),
     "bd_tc_persist_kernel<1>": (
-        543542000, "0f1dbc2f5b303f37",
+        543877080, "cde748c09c00bdc2",
         "ncu, denoise decode, median of 5 launches of `bench.py --only decode`"),
 }
 
