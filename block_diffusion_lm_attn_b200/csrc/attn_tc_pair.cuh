@@ -36,6 +36,10 @@
 namespace bd {
 
 constexpr int kPairThreads = 384;
+// query tiles per half from which the paired kernel runs its EMU variant:
+// measured on B200, training shape (16 tiles, items of ~9 key tiles) 1.5 %
+// faster without, long context (64 tiles, ~32 key tiles) 1.4 % faster with
+constexpr int kPairEmuQtiles = 32;
 constexpr int kPairRegsSoftmax = 208; // setmaxnreg of warpgroups 0 and 1
 constexpr int kPairRegsOther = 88;    // setmaxnreg of warpgroup 2
 static_assert(2 * 128 * kPairRegsSoftmax + 128 * kPairRegsOther <=
@@ -92,8 +96,11 @@ __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
 
 // DH: head dim of the tensors, 128, or 64 / 32 read zero-extended to 128
 // columns (the QKs skip the zero K-steps; the columns of O past DH are never
-// written).
-template <int DH>
+// written).  EMU: a quarter of each tile's exponentials on the FMA pipe
+// (ex2_poly2).  That pays on long work items, where the softmax runs in
+// steady state, and costs on short ones, where the extra instructions land
+// on the item boundaries' critical path; the launch chooses (kPairEmuQtiles).
+template <int DH, bool EMU>
 __global__ void __launch_bounds__(kPairThreads, 1)
     bd_tc_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -409,7 +416,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 tc_fence_after();
                 const bool full = ks >= flo && ks + kTcN <= fhi && ks + kTcN <= khi;
                 const long long jp = jg - 1;
-                ok = softmax_tile<kEmuExp2>(
+                ok = softmax_tile<EMU>(
                     t_s + lane_off, t_o + lane_off, full, sp, ks, khi, sl2, jj >= 1, m_used, l,
                     [&] {
                         return mbar_wait(bar_odone(x, (int)(jp & 1)), (uint32_t)((jp >> 1) & 1),

@@ -54,9 +54,12 @@ bool pair_kernel_usable()
     int u = usable.load();
     if (u < 0) {
         cudaFuncAttributes a;
-        u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel<DH>) == cudaSuccess &&
-             (long long)a.numRegs * bd::kPairThreads >=
-                 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther)
+        cudaFuncAttributes b;
+        const long long need = 2LL * 128 * bd::kPairRegsSoftmax + 128LL * bd::kPairRegsOther;
+        u = (cudaFuncGetAttributes(&a, bd::bd_tc_pair_kernel<DH, true>) == cudaSuccess &&
+             cudaFuncGetAttributes(&b, bd::bd_tc_pair_kernel<DH, false>) == cudaSuccess &&
+             (long long)a.numRegs * bd::kPairThreads >= need &&
+             (long long)b.numRegs * bd::kPairThreads >= need)
                 ? 1
                 : 0;
         usable.store(u);
@@ -226,14 +229,23 @@ bd_status launch_persist_dh(const CUtensorMap &mq, const CUtensorMap &mk,
     return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
 }
 
+template <int DH, bool EMU>
+bd_status launch_pair_emu(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                          const bd::PParams &p, int grid, cudaStream_t st)
+{
+    if (set_smem<bd::bd_tc_pair_kernel<DH, EMU>>(bd::kPairSmemBytes) != BD_OK)
+        return BD_ERR_CUDA;
+    bd::bd_tc_pair_kernel<DH, EMU><<<grid, bd::kPairThreads, bd::kPairSmemBytes, st>>>(mq, mk,
+                                                                                       mv, p);
+    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
 template <int DH>
 bd_status launch_pair(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                       const bd::PParams &p, int grid, cudaStream_t st)
 {
-    if (set_smem<bd::bd_tc_pair_kernel<DH>>(bd::kPairSmemBytes) != BD_OK)
-        return BD_ERR_CUDA;
-    bd::bd_tc_pair_kernel<DH><<<grid, bd::kPairThreads, bd::kPairSmemBytes, st>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+    return p.qtiles >= bd::kPairEmuQtiles ? launch_pair_emu<DH, true>(mq, mk, mv, p, grid, st)
+                                          : launch_pair_emu<DH, false>(mq, mk, mv, p, grid, st);
 }
 
 template <int KIND>
