@@ -145,6 +145,17 @@ def test_fwd_long_context_sampled(bb):
     _fwd_sampled(bd_inputs.FWD_LONG[bb], 800)
 
 
+@pytest.mark.parametrize("d", [64, 32])
+def test_fwd_long_items_at_smaller_head_dims_sampled(d):
+    """From 32 query tiles per half the paired kernel runs its variant with
+    a quarter of the exponentials on the FMA pipe; the long-context rows
+    cover it at head dim 128, this at 64 and 32."""
+    s = bd_inputs.FwdShape("fwd_long_items_d%d" % d, 1, 4, 2, 4096, 16, d, seed=31)
+    assert s.L // 128 >= 32  # the variant's threshold, in query tiles per half
+    assert bd.bd_attn_debug_fwd_kernel(s.Hq, s.Hkv, d) == 2
+    _fwd_sampled(s, 600)
+
+
 def test_fwd_training_shape_invariants():
     """Properties that hold at any size: v = 1 gives out = 1, and the
     result is bit-identical run to run."""
