@@ -179,10 +179,11 @@ BD_API size_t bd_attn_bwd_workspace_bytes(int B, int Hq, int L);
  *                    NULL makes the library use an internal buffer of the
  *                    current device, allocated by the first such call (so
  *                    that call must not be inside a stream capture) and
- *                    never freed, so graphs captured with it stay valid.  Every NULL-workspace call on a device shares
- *                    the current buffer: calls whose kernels may overlap on
- *                    the GPU (two streams without ordering between them)
- *                    race on it and give wrong results -- order them, or
+ *                    never freed, so graphs captured with it stay valid.
+ *                    Every NULL-workspace call on a device shares that
+ *                    buffer: calls whose kernels may overlap on the GPU (two
+ *                    streams without ordering between them) race on it and
+ *                    give wrong results -- order them, or
  *                    pass each stream its own workspace.
  *
  * Errors: BD_ERR_INVALID_ARG for a null or misaligned pointer, any size <= 0,
