@@ -217,8 +217,8 @@ BD_API bd_status bd_attn_decode(const void *q_blk, const void *k_cache,
  * bd_attn_decode computes, with the same arguments, layouts and errors, but
  * takes no workspace: its scratch (bd_attn_decode_workspace_bytes, 19.6 MB
  * for every size) lives in a fixed array of BD_ATTN_NOALLOC_SCRATCH_BYTES
- * bytes compiled into the library's device code.  Every GPU on which the library's kernels are loaded holds that array
- * until the process exits.
+ * bytes compiled into the library's device code.  Every GPU on which the
+ * library's kernels are loaded holds that array until the process exits.
  *
  * - The first call on a device looks up the array's device address (with
  *   that device current) and caches it; make that first call before any
