@@ -610,9 +610,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (!ok)
                 break;
             {
+                // Wait for PV_{jl-1}, then PV_jl.  A parity wait is sound only
+                // while its barrier is at most one phase short, and odone of
+                // PV_jl last completed for PV_{jl-2}, which (issued after QK_jl
+                // in the forward's order) may still run when this warp gets
+                // here.  odone of PV_{jl-1} last completed for PV_{jl-3},
+                // issued before QK_jl and so finished; once PV_{jl-1} is done,
+                // so is PV_{jl-2}.
                 const long long jl = j + sg.nt - 1; // last PV of the segment
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_odone0 + 8 * (jl & 1),
-                                                       (uint32_t)((jl >> 1) & 1), abort_flag));
+                ok = jl < 1 || __all_sync(0xffffffffu,
+                                          mbar_wait(bar_odone0 + 8 * ((jl - 1) & 1),
+                                                    (uint32_t)(((jl - 1) >> 1) & 1), abort_flag));
+                ok = ok && __all_sync(0xffffffffu,
+                                      mbar_wait(bar_odone0 + 8 * (jl & 1),
+                                                (uint32_t)((jl >> 1) & 1), abort_flag));
                 if (!ok)
                     break;
                 tc_fence_after();
