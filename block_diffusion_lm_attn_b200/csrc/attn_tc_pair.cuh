@@ -55,8 +55,8 @@ constexpr int kPairSmemBar = kPairSmemEpi + 8 * 32 * 128;
 constexpr int kPairSmemBytes = kPairSmemBar + 512 + 1024;
 static_assert(kPairSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
-// Work item w of the pair kernel: (batch, head pair) = w / R, cost rank
-// r = w % R (0 = heaviest), as FwdSource with head pairs for heads.
+// Work item w of the pair kernel: (batch, head pair) bp and cost rank r
+// (0 = heaviest) in chunked rank order, as FwdSource with head pairs for heads.
 struct PairSeg {
     int qhead;  // global index (batch * Hq + head) of tile A; tile B is +1
     int qrow0, nrows, kvhead;
@@ -73,8 +73,8 @@ __device__ __forceinline__ long long pair_items(const PParams &p)
 __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
 {
     const int R = 2 * p.qtiles;
-    const int bp = w / R; // batch * (Hq / 2) + pair
-    const int r = w % R;
+    int bp, r; // bp = batch * (Hq / 2) + pair
+    chunked_rank_order(w, p.B * (p.Hq / 2), R, kFwdChunkHeads, bp, r);
     const int idx = p.qtiles - 1 - (r >> 1);
     const int clean = r & 1;
     const int half = p.Hq / 2;
