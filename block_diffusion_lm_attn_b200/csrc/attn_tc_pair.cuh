@@ -52,18 +52,20 @@ constexpr int kPairSmemK = kPairSmemQ + 2 * kTileBytes; // 2 stages
 constexpr int kPairSmemV = kPairSmemK + 2 * kTileBytes; // 2 stages
 constexpr int kPairSmemEpi = kPairSmemV + 2 * kTileBytes; // 8 warps x 4 KB
 constexpr int kPairSmemBar = kPairSmemEpi + 8 * 32 * 128;
-constexpr int kPairSmemBytes = kPairSmemBar + 512 + 1024;
+constexpr int kPairSmemSeg = kPairSmemBar + 512; // 4 decoded work items (PairSeg)
+constexpr int kPairSmemBytes = kPairSmemSeg + 4 * 64 + 1024;
 static_assert(kPairSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
 // Work item w of the pair kernel: (batch, head pair) bp and cost rank r
 // (0 = heaviest) in chunked rank order, as FwdSource with head pairs for heads.
-struct PairSeg {
+struct alignas(16) PairSeg {
     int qhead;  // global index (batch * Hq + head) of tile A; tile B is +1
     int qrow0, nrows, kvhead;
     int lo0, hi0, lo1, hi1;
     int flo0, fhi0, flo1, fhi1;
     int n0, nt;
 };
+static_assert(sizeof(PairSeg) <= 64, "a decoded work item takes one 64-byte slot");
 
 __device__ __forceinline__ long long pair_items(const PParams &p)
 {
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const uint32_t bar_ifull0 = bar0 + 168;  // 4: work item published
     const uint32_t bar_iempty0 = bar0 + 200; // 4: work item read by all roles
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 256);
+    PairSeg *seg_ring = reinterpret_cast<PairSeg *>(sbase + kPairSmemSeg);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kPairSmemBar + 384);
     volatile uint32_t *tmem_slot =
         reinterpret_cast<volatile uint32_t *>(sbase + kPairSmemBar + 392);
@@ -169,9 +172,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
     PairSeg sg;
     // Next item of this CTA, identical for every role: the Q/K producer
-    // takes it from the launch's global counter and publishes it in
-    // item_ring[si % 4]; the other roles read it there.
-    auto next_seg = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
+    // takes it from the launch's global counter, decodes it (pair_item, a
+    // few integer divisions: ~1800 cycles of one warp, measured) and
+    // publishes index and decoded item in slot si % 4; the other roles copy
+    // the decoded item, so the divisions stay off the softmax and MMA paths.
+    // arrive: 0 none, 1 this thread, 2 the whole (converged) warp, through
+    // lane 0 once every lane has read the slot.
+    auto next_seg = [&](int si, bool producer, bool &ok, int arrive = 1) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -182,19 +189,30 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < pair_items(p) ? (int)t : -1;
+            if (w >= 0) {
+                pair_item(p, w, sg);
+                seg_ring[slot] = sg;
+            }
             item_ring[slot] = w;
             mbar_arrive(bar_ifull0 + 8 * slot);
         } else {
-            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+            ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag);
+            if (arrive == 2) // one outcome for the warp before its __syncwarp
+                ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
                 return false;
             w = item_ring[slot];
-            if (arrive)
+            if (w >= 0)
+                sg = seg_ring[slot];
+            if (arrive == 2) {
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0)
+                    mbar_arrive(bar_iempty0 + 8 * slot);
+            } else if (arrive == 1) {
                 mbar_arrive(bar_iempty0 + 8 * slot);
+            }
         }
-        if (w < 0)
-            return false;
-        pair_item(p, w, sg);
-        return true;
+        return w >= 0;
     };
     auto key_start = [&](int it) {
         return it < sg.n0 ? sg.lo0 + it * kTcN : sg.lo1 + (it - sg.n0) * kTcN;
@@ -321,7 +339,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                                       abort_flag);
             };
             for (;;) {
-                const bool got = next_seg(si, false, ok, lane == 0);
+                const bool got = next_seg(si, false, ok, 2);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!got || !ok)
                     break;
@@ -447,6 +465,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const float lse_v = (l > 0.f) ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
             const size_t head_row0 = (size_t)(sg.qhead + x) * 2 * p.L + sg.qrow0;
             const uint32_t epi = base + kPairSmemEpi + (uint32_t)warp * (32 * 128);
+            // O in one load (one TMEM round trip, not one per 32 columns);
+            // once it is in registers the next item's first PV may overwrite it
+            uint32_t ov[kTcD];
+            if constexpr (DH > 64)
+                tmem_ld32x4_wait(t_o + lane_off, t_o + lane_off + 32, t_o + lane_off + 64,
+                                 t_o + lane_off + 96, ov, ov + 32, ov + 64, ov + 96);
+            else if constexpr (DH > 32)
+                tmem_ld32x2_wait(t_o + lane_off, t_o + lane_off + 32, ov, ov + 32);
+            else
+                tmem_ld32_wait(t_o + lane_off, ov);
+            tc_fence_before();
+            mbar_arrive(bar_ofree(x));
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 if (h * 64 >= DH) // O columns past the head dim are not output
@@ -456,8 +486,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const int q4 = 2 * h + q;
                     if (q4 * 32 >= DH)
                         break;
-                    uint32_t o[32];
-                    tmem_ld32_wait(t_o + lane_off + q4 * 32, o);
+                    const uint32_t *o = ov + q4 * 32;
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
                         const uint32_t cch = (uint32_t)(q * 4 + i / 8);
@@ -490,8 +519,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             }
             if (row < sg.nrows)
                 p.lse[head_row0 + row] = lse_v;
-            tc_fence_before();
-            mbar_arrive(bar_ofree(x));
             j += sg.nt;
             ++si;
         }
