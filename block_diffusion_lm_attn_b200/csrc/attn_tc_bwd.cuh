@@ -40,6 +40,7 @@ struct BParams {
     int B, Hq, Hkv, L, b;
     int qtiles;     // 128-row tiles per half
     int sched_slot; // counter pair of this launch
+    int chunk_q;    // dQ: heads per chunk of the work list (as PParams::chunk)
     float scale, scale_log2;
 };
 
@@ -771,6 +772,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     PParams fp = {};
     fp.B = p.B; fp.Hq = p.Hq; fp.Hkv = p.Hkv; fp.L = p.L; fp.b = p.b;
     fp.qtiles = p.qtiles;
+    fp.chunk = p.chunk_q;
     Seg sg;
     auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
         const int slot = si & 3;

@@ -37,9 +37,12 @@ namespace bd {
 
 constexpr int kPairThreads = 384;
 // query tiles per half from which the paired kernel runs its EMU variant:
-// measured on B200, training shape (16 tiles, items of ~9 key tiles) 1.5 %
-// faster without, long context (64 tiles, ~32 key tiles) 1.4 % faster with
-constexpr int kPairEmuQtiles = 32;
+// measured on B200, the training shape (16 tiles, items of ~9 key tiles) 3 %
+// faster with, the long context (64 tiles, ~32 key tiles) 1.4 % faster with.
+// (Before each item was decoded once, in the producer, the training shape
+// was 1.5 % faster without: the extra instructions then landed on the item
+// boundaries' critical path.)
+constexpr int kPairEmuQtiles = 16;
 constexpr int kPairRegsSoftmax = 208; // setmaxnreg of warpgroups 0 and 1
 constexpr int kPairRegsOther = 88;    // setmaxnreg of warpgroup 2
 static_assert(2 * 128 * kPairRegsSoftmax + 128 * kPairRegsOther <=
@@ -76,7 +79,7 @@ __device__ __forceinline__ void pair_item(const PParams &p, int w, PairSeg &sg)
 {
     const int R = 2 * p.qtiles;
     int bp, r; // bp = batch * (Hq / 2) + pair
-    chunked_rank_order(w, p.B * (p.Hq / 2), R, kFwdChunkHeads, bp, r);
+    chunked_rank_order(w, p.B * (p.Hq / 2), R, p.chunk, bp, r);
     const int idx = p.qtiles - 1 - (r >> 1);
     const int clean = r & 1;
     const int half = p.Hq / 2;

@@ -47,6 +47,7 @@ struct PParams {
     int row_tiles; // decode: 128-row query tiles per unit
     int rows_unit; // decode: query rows per (sequence, kv-head) = group * b
     int sched_slot; // fwd: counter pair of this launch (0 .. kSchedSlots-1)
+    int chunk;      // fwd: heads (head pairs in the paired kernel) per chunk of the work list
     float scale_log2;
 };
 
@@ -86,10 +87,11 @@ __device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap, int 
 // The work items are handed out dynamically: the TMA producer of each CTA
 // takes the next item index from a global counter and passes it to the MMA
 // and softmax roles through a 4-entry ring in shared memory.  The heads are
-// taken in chunks of kFwdChunkHeads; inside a chunk the list runs rank by
-// rank (every head's heaviest query tile, then every head's next ...).  The
-// CTAs running at any moment then share the K/V of a few kv-heads in L2, and
-// the list ends on the lightest tiles of its last chunk.  Head by head (one
+// taken in chunks of p.chunk (the host sizes a chunk so that its K/V fit in
+// half of L2); inside a chunk the list runs rank by rank (every head's
+// heaviest query tile, then every head's next ...).  The CTAs running at any
+// moment then share the K/V of the chunk in L2, and the list ends on the
+// lightest tiles of its last chunk.  Head by head (one
 // head's tiles heaviest first, then the next head's) the heaviest tiles of
 // the last heads were handed out near the end: a list-scheduling model of
 // the training shape puts the time lost to the tail at 7 % for the paired
@@ -97,7 +99,6 @@ __device__ __forceinline__ int decode_unit_tiles(int len, int b, int S_cap, int 
 // one of kSchedSlots counter pairs (rotating on the host); the last CTA of a
 // launch to finish resets its pair.
 constexpr int kSchedSlots = 64;
-constexpr int kFwdChunkHeads = 16; // heads (pairs in the paired kernel) per chunk
 
 // Position w of a list of G groups x R ranks that runs chunk by chunk (C
 // groups a chunk, the last one possibly smaller) and rank by rank inside a
@@ -151,7 +152,7 @@ struct FwdSource {
     {
         const int R = 2 * p.qtiles;
         int bh, r;
-        chunked_rank_order(w, p.B * p.Hq, R, kFwdChunkHeads, bh, r);
+        chunked_rank_order(w, p.B * p.Hq, R, p.chunk, bh, r);
         const int idx = p.qtiles - 1 - (r >> 1);
         const int clean = r & 1; // noisy tile k is one K/V tile heavier
         sg.qrow0 = (clean ? p.L : 0) + idx * kTcM;
