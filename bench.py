@@ -63,11 +63,10 @@ KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
     "bd_tc_pair_kernel": (
-        301932032, "dc3687d38843913c",
-        "ncu, training-shape forward (its no-polynomial variant), 4th launch of "
-        "`bench.py --only fwd`"),
+        313629952, "1d2c5e26761345f8",
+        "ncu, training-shape forward, 4th launch of `bench.py --only fwd`"),
     "bd_tc_persist_kernel<1>": (
-        544153232, "dc3687d38843913c",
+        543802328, "1d2c5e26761345f8",
         "ncu, denoise decode, median of 5 launches of `bench.py --only decode`"),
 }
 

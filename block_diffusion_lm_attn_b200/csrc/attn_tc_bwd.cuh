@@ -685,7 +685,9 @@ constexpr int kDqVStages = 2;
 constexpr int kDqSmemK = kDqSmemDO + kTileBytes;               // K stages
 constexpr int kDqSmemV = kDqSmemK + kDqKStages * kTileBytes;  // V stages
 constexpr int kDqSmemBar = kDqSmemV + kDqVStages * kTileBytes;
-constexpr int kDqSmemBytes = kDqSmemBar + 512 + 1024;
+constexpr int kDqSmemSeg = kDqSmemBar + 512; // 4 decoded work items (Seg)
+constexpr int kDqSmemBytes = kDqSmemSeg + 4 * 128 + 1024;
+static_assert(sizeof(Seg) <= 128, "a decoded work item takes one 128-byte slot");
 static_assert(kDqSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
 // Roles: warps 0-7 compute dS (warp w: query rows of TMEM lane quarter
@@ -723,6 +725,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto bar_vempty = [&](int s) { return bar0 + 152 + 16 * kDqKStages + 8 * kDqVStages + 8 * s; };
     static_assert(152 + 16 * kDqKStages + 16 * kDqVStages <= 256, "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 256);
+    Seg *seg_ring = reinterpret_cast<Seg *>(sbase + kDqSmemSeg);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kDqSmemBar + 384);
     volatile uint32_t *tmem_slot =
         reinterpret_cast<volatile uint32_t *>(sbase + kDqSmemBar + 392);
@@ -774,7 +777,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fp.qtiles = p.qtiles;
     fp.chunk = p.chunk_q;
     Seg sg;
-    auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
+    // As in the paired forward: the producer decodes the item it claims and
+    // publishes it in slot si % 4; the other roles copy it (arrive: 0 none,
+    // 1 this thread, 2 the converged warp through lane 0).
+    auto next_item = [&](int si, bool producer, bool &ok, int arrive = 1) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -785,19 +791,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < FwdSource::items(fp) ? (int)t : -1;
+            if (w >= 0) {
+                FwdSource::item(fp, w, sg);
+                seg_ring[slot] = sg;
+            }
             item_ring[slot] = w;
             mbar_arrive(bar_ifull0 + 8 * slot);
         } else {
-            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+            ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag);
+            if (arrive == 2) // one outcome for the warp before its __syncwarp
+                ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
                 return false;
             w = item_ring[slot];
-            if (arrive)
+            if (w >= 0)
+                sg = seg_ring[slot];
+            if (arrive == 2) {
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0)
+                    mbar_arrive(bar_iempty0 + 8 * slot);
+            } else if (arrive == 1) {
                 mbar_arrive(bar_iempty0 + 8 * slot);
+            }
         }
-        if (w < 0)
-            return false;
-        FwdSource::item(fp, w, sg);
-        return true;
+        return w >= 0;
     };
     auto key_start = [&](int t) {
         return t < sg.n0 ? sg.lo0 + t * kTcN : sg.lo1 + (t - sg.n0) * kTcN;
@@ -906,7 +923,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_commit_p(bar_kempty((int)(jg % kDqKStages)), ld);
             };
             for (;;) {
-                const bool got = next_item(si, false, ok, lane == 0);
+                const bool got = next_item(si, false, ok, 2);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!got || !ok)
                     break;
