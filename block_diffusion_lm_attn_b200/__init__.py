@@ -191,6 +191,16 @@ def bd_attn_debug_set_grid(ctas):
     return fn(ctas)
 
 
+def bd_attn_debug_set_chunk(groups):
+    """Test hook (include/bd_attn_debug.h): fix the chunk size of the work
+    lists at `groups` heads / head pairs / kv-head groups (0 restores the
+    defaults)."""
+    fn = load().bd_attn_debug_set_chunk
+    fn.restype = ctypes.c_int
+    fn.argtypes = [ctypes.c_int]
+    return fn(groups)
+
+
 # ---------------------------------------------------------------------------
 # torch-tensor conveniences
 

@@ -41,6 +41,7 @@ struct BParams {
     int qtiles;     // 128-row tiles per half
     int sched_slot; // counter pair of this launch
     int chunk_q;    // dQ: heads per chunk of the work list (as PParams::chunk)
+    int chunk_kv;   // dK/dV: (batch, kv-head) groups per chunk of the clean key tiles
     float scale, scale_log2;
 };
 
@@ -168,12 +169,13 @@ static_assert(kBwdSub == 128, "the dK/dV compute warps take 64 query columns eac
 // 0 .. qtiles-1 are the clean key tiles, idx ascending (heaviest first: a
 // clean key tile idx is seen by 2 (qtiles - idx) query tiles of each q-head);
 // ranks qtiles .. 2 qtiles-1 the noisy ones (one query tile each).  The list
-// holds every clean item first, kBwdChunkGroups groups at a time in rank
-// order (so the running CTAs share the Q and dO of a few groups in L2), and
-// then every noisy item.  Group by group, the heaviest items of the last
-// groups came near the end of the list: a list-scheduling model of the
-// training shape lost 25 % of the pass to its tail, against about 1 % this
-// way (an item is up to half of a CTA's average load).
+// holds every clean item first, p.chunk_kv groups at a time (by default
+// kBwdChunkGroups) in rank order, so that the running CTAs share the Q and
+// dO of a few groups in L2, and then every noisy item.  Group by group, the
+// heaviest items of the last groups came near the end of the list: a
+// list-scheduling model of the training shape lost 25 % of the pass to its
+// tail, against about 1 % this way (an item is up to half of a CTA's average
+// load).
 struct KvItem {
     int kvhead;       // batch * Hkv + kv-head
     int qhead0;       // batch * Hq + first q-head of the group
@@ -195,7 +197,7 @@ __device__ __forceinline__ void kv_item(const BParams &p, int w, KvItem &it)
     const int nclean = NG * p.qtiles;
     int bg, r;
     if (w < nclean) {
-        chunked_rank_order(w, NG, p.qtiles, kBwdChunkGroups, bg, r);
+        chunked_rank_order(w, NG, p.qtiles, p.chunk_kv, bg, r);
     } else {
         r = p.qtiles + (w - nclean) / NG;
         bg = (w - nclean) % NG;

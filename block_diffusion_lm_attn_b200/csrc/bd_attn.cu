@@ -98,8 +98,14 @@ int persistent_grid()
 // heaviest rank first, so the larger it is, the lighter the items that end
 // the list (a list-scheduling model of the training shape: 98.2 % of the
 // balanced time with 16 head pairs a chunk, 99.5 % with 32 or more).
+// Chunk size set by bd_attn_debug_set_chunk (0: the defaults).
+std::atomic<int> g_chunk_fixed{0};
+
 int list_chunk(long long bytes_per_group, long long groups)
 {
+    const int fixed = g_chunk_fixed.load();
+    if (fixed > 0)
+        return (int)std::max(1LL, std::min((long long)fixed, groups));
     constexpr long long kBudget = 64LL << 20;
     const long long c = bytes_per_group > 0 ? kBudget / bytes_per_group : groups;
     return (int)std::max(1LL, std::min(c, groups));
@@ -478,6 +484,8 @@ bd_status bd_attn_bwd(const void *q, const void *k, const void *v,
     p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.L = L; p.b = b;
     p.qtiles = (int)cdiv(L, bd::kTcM);
     p.chunk_q = list_chunk(8LL * L * d / (Hq / Hkv), (long long)B * Hq);
+    const int fixed = g_chunk_fixed.load();
+    p.chunk_kv = fixed > 0 ? fixed : bd::kBwdChunkGroups;
     p.scale = scale;
     p.scale_log2 = scale * bd::kLog2e;
 
@@ -686,6 +694,14 @@ bd_status bd_attn_debug_set_grid(int ctas)
     if (ctas < 0 || ctas > kMaxGrid)
         return BD_ERR_INVALID_ARG;
     g_grid_cap.store(ctas);
+    return BD_OK;
+}
+
+bd_status bd_attn_debug_set_chunk(int groups)
+{
+    if (groups < 0)
+        return BD_ERR_INVALID_ARG;
+    g_chunk_fixed.store(groups);
     return BD_OK;
 }
 

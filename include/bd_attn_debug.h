@@ -42,6 +42,19 @@ BD_API bd_status bd_attn_debug_inject_fault(int kind);
 BD_API bd_status bd_attn_debug_set_grid(int ctas);
 
 /*
+ * Fixes the chunk size of the persistent kernels' work lists for every later
+ * launch from any thread: `groups` heads (head pairs in the paired forward
+ * kernel) per chunk of the forward and dQ lists, and `groups` (batch,
+ * kv-head) groups per chunk of the clean key tiles in the dK/dV list.  Each
+ * list runs chunk by chunk, heaviest item first inside a chunk, so tests can
+ * run several chunks and a ragged last one on small sizes.  groups = 0
+ * restores the default (forward and dQ: as many as keep the chunk's K/V
+ * within 64 MB; dK/dV: 8).  Results are the same for any chunk size up to
+ * rounding order.  Returns BD_OK, or BD_ERR_INVALID_ARG for groups < 0.
+ */
+BD_API bd_status bd_attn_debug_set_chunk(int groups);
+
+/*
  * Which kernel bd_attn_fwd runs for these sizes on the current device:
  * 2 = tcgen05 kernel with two query heads of a GQA group per CTA (even group
  * size), 1 = tcgen05 kernel with one query tile per CTA (odd group size, or

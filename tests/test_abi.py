@@ -131,6 +131,8 @@ def test_grid_hook_rejects_out_of_range(lib):
     assert bd.bd_attn_debug_set_grid(-1) == bd.BD_ERR_INVALID_ARG
     assert bd.bd_attn_debug_set_grid(149) == bd.BD_ERR_INVALID_ARG
     assert bd.bd_attn_debug_set_grid(0) == bd.BD_OK
+    assert bd.bd_attn_debug_set_chunk(-1) == bd.BD_ERR_INVALID_ARG
+    assert bd.bd_attn_debug_set_chunk(0) == bd.BD_OK
 
 
 def test_cache_and_sprint_reject_bad_arguments(lib):

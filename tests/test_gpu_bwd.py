@@ -97,6 +97,25 @@ def test_bwd_at_grid_sizes(ctas):
         check_grad(got, ref, (n, ctas))
 
 
+@pytest.mark.parametrize("chunk", [1, 3])
+def test_bwd_chunked_work_lists(chunk):
+    """Both passes' work lists run chunk by chunk with several chunks and a
+    ragged last one (dK/dV: 4 groups; dQ: 8 heads), on 37 CTAs."""
+    B, Hq, Hkv, L, b, d = 2, 4, 2, 256, 16, 128
+    q, k, v, do = _inputs(B, Hq, Hkv, L, d, seed=40 + chunk)
+    s = 1 / math.sqrt(d)
+    assert bd.bd_attn_debug_set_chunk(chunk) == bd.BD_OK
+    assert bd.bd_attn_debug_set_grid(37) == bd.BD_OK
+    try:
+        dq, dk, dv = _gpu_grads(q, k, v, do, L, b, s)
+    finally:
+        bd.bd_attn_debug_set_grid(0)
+        bd.bd_attn_debug_set_chunk(0)
+    rq, rk, rv = backward.fwd_bwd(q, k, v, do, L, b, s)
+    for got, ref, n in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        check_grad(got, ref, (n, chunk))
+
+
 def test_bwd_training_shape_sampled_groups():
     """The training shape (B=4, Hq=32, Hkv=8, L=2048, b=32, keys x 0.5) in
     the launch configuration the benchmark times; the oracle computes two

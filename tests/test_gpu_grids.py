@@ -27,6 +27,7 @@ def _lib():
     assert torch.cuda.is_available()
     yield
     assert bd.bd_attn_debug_set_grid(0) == bd.BD_OK
+    assert bd.bd_attn_debug_set_chunk(0) == bd.BD_OK
 
 
 def check(out, lse, ro, rl, what):
@@ -53,6 +54,24 @@ def test_fwd_at_grid(ctas):
         assert bd.device_status() == bd.BD_OK
         ro, rl = oracle.fwd(q, k, v, L, b, 1 / math.sqrt(d))
         check(out, lse, ro, rl, (ctas, B, Hq, Hkv, L, b))
+
+
+@pytest.mark.parametrize("chunk", [1, 3])
+def test_fwd_chunked_work_list(chunk):
+    """The forward's work list run chunk by chunk (heaviest item first inside
+    a chunk) with several chunks and a ragged last one: on the paired kernel
+    (4 and 12 head pairs) and on the one-tile kernel (6 heads of an odd
+    group), with a few CTAs so that items of different chunks overlap."""
+    assert bd.bd_attn_debug_set_chunk(chunk) == bd.BD_OK
+    assert bd.bd_attn_debug_set_grid(37) == bd.BD_OK
+    for (B, Hq, Hkv, L, b) in [(2, 4, 2, 200, 8), (3, 8, 2, 256, 32), (2, 3, 1, 200, 8)]:
+        d = 128
+        q, k, v = bd_inputs.fwd_inputs(B, Hq, Hkv, L, d, seed=chunk + 7 * L + B)
+        out, lse = bd.fwd(q.cuda(), k.cuda(), v.cuda(), L, b, 1 / math.sqrt(d))
+        torch.cuda.synchronize()
+        assert bd.device_status() == bd.BD_OK
+        ro, rl = oracle.fwd(q, k, v, L, b, 1 / math.sqrt(d))
+        check(out, lse, ro, rl, (chunk, B, Hq, Hkv, L, b))
 
 
 DEC_CASES = [
