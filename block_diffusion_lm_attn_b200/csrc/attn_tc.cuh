@@ -67,7 +67,8 @@ constexpr int kSmemV = kSmemK + kTcStages * kTileBytes;
 // epilogue staging: per softmax warp, its 32 output rows of 256 bytes
 constexpr int kSmemEpi = kSmemV + kTcStages * kTileBytes;
 constexpr int kSmemBar = kSmemEpi + 4 * 32 * 256;
-constexpr int kTcSmemBytes = kSmemBar + 512 + 1024; // + alignment slack
+constexpr int kSmemSeg = kSmemBar + 512;                // 4 decoded work items, 128 B each
+constexpr int kTcSmemBytes = kSmemSeg + 4 * 128 + 1024; // + alignment slack
 static_assert(kTcSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
 // ---------------------------------------------------------------------------

@@ -63,6 +63,7 @@ struct Seg {
     int last_cta;       // decode: CTA holding the unit's last tile (cut
                         // units that start in this CTA's range), else -1
 };
+static_assert(sizeof(Seg) <= 128, "a decoded work item takes one 128-byte slot");
 
 // Keys a decode row may see past the prefix: the block itself in modes 0
 // and 1, nothing in mode 2 (cross-attention to the prefix only).
@@ -315,6 +316,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     static_assert(8 * (1 + 2 * kTcStages) + 16 * kSBufs + 16 + 8 + 16 + 8 + 8 + 64 <= 256,
                   "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kSmemBar + 256);
+    Seg *seg_ring = reinterpret_cast<Seg *>(sbase + kSmemSeg);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kSmemBar + 384);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + kSmemBar + 392);
 
@@ -374,9 +376,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
 
     // Next segment of this CTA, identical for every role.  Training/prefill:
-    // the producer takes the next item from the global counter and publishes
-    // it in item_ring[si % 4]; the other roles read it there.  Decode: each
-    // role walks its static stream-K range.
+    // the producer takes the next item from the global counter, decodes it
+    // (FwdSource::item: a few integer divisions) and publishes index and
+    // decoded item in slot si % 4; the other roles copy it from there.
+    // Decode: each role walks its static stream-K range.
     auto next_seg = [&](int si, bool producer, bool &ok) -> bool {
         if constexpr (KIND == 1) {
             return src.next(p, sg);
@@ -391,18 +394,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < FwdSource::items(p) ? (int)t : -1;
+            if (w >= 0) {
+                FwdSource::item(p, w, sg);
+                seg_ring[slot] = sg;
+            }
             item_ring[slot] = w;
             mbar_arrive(bar_ifull0 + 8 * slot);
         } else {
             if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
                 return false;
             w = item_ring[slot];
+            if (w >= 0)
+                sg = seg_ring[slot];
             mbar_arrive(bar_iempty0 + 8 * slot);
         }
-        if (w < 0)
-            return false;
-        FwdSource::item(p, w, sg);
-        return true;
+        return w >= 0;
         }
     };
 
