@@ -63,10 +63,10 @@ KERNEL_SOURCES = ("attn_tc.cuh", "attn_tc_persist.cuh", "attn_tc_pair.cuh",
 TRAFFIC = {
     # kernel: (bytes per launch, source digest at capture time, capture)
     "bd_tc_pair_kernel": (
-        313629952, "1d2c5e26761345f8",
+        313214208, "1c71ede8fd6fbc4f",
         "ncu, training-shape forward, 4th launch of `bench.py --only fwd`"),
     "bd_tc_persist_kernel<1>": (
-        543802328, "1d2c5e26761345f8",
+        543586768, "1c71ede8fd6fbc4f",
         "ncu, denoise decode, median of 5 launches of `bench.py --only decode`"),
 }
 
