@@ -176,7 +176,7 @@ static_assert(kBwdSub == 128, "the dK/dV compute warps take 64 query columns eac
 // list-scheduling model of the training shape lost 25 % of the pass to its
 // tail, against about 1 % this way (an item is up to half of a CTA's average
 // load).
-struct KvItem {
+struct alignas(16) KvItem {
     int kvhead;       // batch * Hkv + kv-head
     int qhead0;       // batch * Hq + first q-head of the group
     int krow0, nkeys; // first key row (of 2L), valid keys (<= 128)
@@ -185,6 +185,7 @@ struct KvItem {
     int n0, n1;       // steps of range 0 / range 1 per q-head
     int nt;           // steps of the item (all q-heads)
 };
+static_assert(sizeof(KvItem) <= 64, "a decoded work item takes one 64-byte slot");
 
 __device__ __forceinline__ long long kv_items(const BParams &p)
 {
@@ -242,7 +243,8 @@ constexpr int kKvStageBytes = 2 * kSubBytes;
 constexpr int kKvSmemRows = kKvSmemRing + kKvStages * kKvStageBytes; // lse2, D
 constexpr int kKvRowsBytes = 2 * kBwdSub * 4;
 constexpr int kKvSmemBar = kKvSmemRows + kKvStages * kKvRowsBytes;
-constexpr int kKvSmemBytes = kKvSmemBar + 512 + 1024;
+constexpr int kKvSmemSeg = kKvSmemBar + 512; // 4 decoded work items (KvItem)
+constexpr int kKvSmemBytes = kKvSmemSeg + 4 * 64 + 1024;
 static_assert(kKvStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(kKvSmemBytes <= 227 * 1024, "more shared memory than a CTA may have");
 
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t bar_iempty0 = bar1 + 88; // 4: work item read by all roles
     static_assert(16 + 16 * kKvStages + 120 <= 256, "barriers overlap the item ring");
     volatile int *item_ring = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 256);
+    KvItem *kv_ring = reinterpret_cast<KvItem *>(sbase + kKvSmemSeg);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + kKvSmemBar + 384);
     volatile uint32_t *tmem_slot =
         reinterpret_cast<volatile uint32_t *>(sbase + kKvSmemBar + 392);
@@ -333,7 +336,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_dv = tmem, t_dk = tmem + 128, t_st = tmem + 256, t_dp = tmem + 384;
 
     KvItem it;
-    auto next_item = [&](int si, bool producer, bool &ok, bool arrive = true) -> bool {
+    // As in the forward: the producer decodes the item it claims and
+    // publishes it in slot si % 4; the other roles copy it (arrive: 0 none,
+    // 1 this thread, 2 the converged warp through lane 0).
+    auto next_item = [&](int si, bool producer, bool &ok, int arrive = 1) -> bool {
         const int slot = si & 3;
         int w;
         if (producer) {
@@ -344,19 +350,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 sched_claim(p.sched_slot);
             const unsigned int t = atomicAdd(&g_sched_next[p.sched_slot], 1u);
             w = (long long)t < kv_items(p) ? (int)t : -1;
+            if (w >= 0) {
+                kv_item(p, w, it);
+                kv_ring[slot] = it;
+            }
             item_ring[slot] = w;
             mbar_arrive(bar_ifull0 + 8 * slot);
         } else {
-            if (!(ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag)))
+            ok = mbar_wait(bar_ifull0 + 8 * slot, (uint32_t)((si >> 2) & 1), abort_flag);
+            if (arrive == 2) // one outcome for the warp before its __syncwarp
+                ok = __all_sync(0xffffffffu, ok);
+            if (!ok)
                 return false;
             w = item_ring[slot];
-            if (arrive)
+            if (w >= 0)
+                it = kv_ring[slot];
+            if (arrive == 2) {
+                __syncwarp();
+                if ((threadIdx.x & 31) == 0)
+                    mbar_arrive(bar_iempty0 + 8 * slot);
+            } else if (arrive == 1) {
                 mbar_arrive(bar_iempty0 + 8 * slot);
+            }
         }
-        if (w < 0)
-            return false;
-        kv_item(p, w, it);
-        return true;
+        return w >= 0;
     };
 
     if (warp == kBwdProducerWarp) {
@@ -374,7 +391,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!got)
                 break;
             if (lane != 0)
-                kv_item(p, item_ring[si & 3], it);
+                it = kv_ring[si & 3];
             if (lane == 0) {
                 // K, V of item si - 1 are no longer read
                 if (si >= 1 && !(ok = mbar_wait(bar_kvfree, (uint32_t)((si - 1) & 1), abort_flag)))
@@ -483,7 +500,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             };
             for (;;) {
-                const bool got = next_item(si, false, ok, lane == 0);
+                const bool got = next_item(si, false, ok, 2);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!got || !ok)
                     break;
